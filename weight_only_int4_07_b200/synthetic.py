@@ -1,0 +1,61 @@
+"""Seeded synthetic inputs for the W4A16 linear layer.
+
+This module only draws random numbers: it holds none of the layer's arithmetic (no
+quantization, packing, dequantization or products). Both the FP64 oracle's checks and the CUDA
+path take their inputs from here. Every generator is seeded (numpy PCG64) and returns uint16
+bit patterns of the 16-bit float type, so the two sides see identical bits.
+
+Distributions follow the workloads the layer is measured on:
+  * weights ~ N(0, 0.02) in fp16;
+  * weights ~ N(0, 0.02) with a fixed fraction of entries (chosen by a seeded permutation)
+    multiplied by a constant (outliers);
+  * weights ~ 0.02 * Student-t(nu=5) in fp16;
+  * activations ~ N(0, 1) in fp16 or bf16.
+"""
+import numpy as np
+import torch
+
+F16 = 0
+BF16 = 1
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _to_bits(x32: np.ndarray, dtype: int) -> np.ndarray:
+    """Round float32 samples to the 16-bit input type and return the bit patterns."""
+    if dtype == F16:
+        return np.ascontiguousarray(x32.astype(np.float16)).view(np.uint16)
+    t = torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def weights_normal(K, N, seed, std=0.02):
+    return _to_bits(_rng(seed).standard_normal((K, N), dtype=np.float32) * np.float32(std), F16)
+
+
+def weights_outliers(K, N, seed, std=0.02, frac=0.001, mult=20.0):
+    rng = _rng(seed)
+    w = rng.standard_normal((K, N), dtype=np.float32) * np.float32(std)
+    n_out = int(round(frac * K * N))
+    idx = rng.permutation(K * N)[:n_out]
+    w.reshape(-1)[idx] *= np.float32(mult)
+    return _to_bits(w, F16)
+
+
+def weights_student_t(K, N, seed, nu=5.0, scale=0.02):
+    w = _rng(seed).standard_t(nu, size=(K, N)).astype(np.float32) * np.float32(scale)
+    return _to_bits(w, F16)
+
+
+def activations(M, K, seed, dtype=F16, std=1.0):
+    return _to_bits(_rng(seed).standard_normal((M, K), dtype=np.float32) * np.float32(std), dtype)
+
+
+def column_sample(N, count, seed):
+    """A seeded sample of output columns that always holds the first and the last column."""
+    rng = _rng(seed)
+    cols = set(int(c) for c in rng.choice(N, size=min(count, N), replace=False))
+    cols.update({0, N - 1})
+    return np.array(sorted(cols), dtype=np.int64)
