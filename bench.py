@@ -1,0 +1,579 @@
+#!/usr/bin/env python
+"""W4A16 GEMM throughput on B200: HBM GB/s at M=1 and TFLOPS at M=256, against the roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (N=1 line): the decode linears of a 32-layer Llama-3-8B-shaped model for one token,
+M = 1: per layer (K, N) = (4096, 6144) qkv, (4096, 4096) o, (4096, 28672) gate+up,
+(14336, 4096) down; g128 asymmetric INT4; fp16 activations ~ N(0, 1); weights ~ N(0, 0.02).
+Four weight matrices are drawn and quantized, and each is copied into 32 distinct device
+buffers: one step streams 3.63 GB of packed weights, so L2 (126 MB) cannot serve repeats.
+A step is the 128 GEMMs of one token, replayed from a CUDA graph.
+
+Printed (rank 0, one JSON line): value = algorithmic bytes of all ranks' steps / max-over-ranks
+device time (GB/s); e2e = the same through the Python API with the step's activations copied
+from pinned host memory and its outputs read back; roofline of the dominant kernel; the FP64
+oracle's throughput on the host cores (cpu_baseline); clocks sampled during the timed region;
+and an M = 256 measurement on the (8192, 28672) sweep layer (TFLOPS).
+
+N > 1 (torchrun): weak scaling, every rank runs its own replica of the workload; no collective
+on the data path (NCCL carries only the barrier and the max of the timings).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+LLAMA8B_LINEARS = (("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672),
+                   ("down", 14336, 4096))
+LAYERS = 32
+GROUP = 128
+SYM = 0
+SWEEP_K, SWEEP_N, SWEEP_M = 8192, 28672, 256
+METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=256, as % of B200 roofline"
+
+
+# ----------------------------------------------------------------------------- work model
+def algorithmic_bytes(M, K, N, group=GROUP, sym=SYM, act_bytes=2, out_bytes=2):
+    """Bytes a W4A16 GEMM must move at least once: codes 0.5 B/weight, an fp16 scale per
+    group, an INT4 zero per group (asymmetric), the activations and the output."""
+    codes = K * N // 2
+    scales = 2 * N * (K // group)
+    zeros = 0 if sym else N * (K // group) // 2
+    return codes + scales + zeros + act_bytes * M * K + out_bytes * M * N
+
+
+def gemm_flops(M, K, N):
+    return 2 * M * N * K
+
+
+def step_time_model(params, bits_per_weight, bytes_per_s, flops_per_s, batch):
+    """Roofline time of one decode step: max(weight bytes / bandwidth, 2 * params * batch / flops)
+    ("INT8 vs INT4 Quantization, in depth", section "Worked example: where the lines cross")."""
+    t_mem = params * bits_per_weight / 8 / bytes_per_s
+    t_math = 2 * params * batch / flops_per_s
+    return max(t_mem, t_math), t_mem, t_math
+
+
+def crossover_batch(params, bits_per_weight, bytes_per_s, flops_per_s):
+    """Batch at which the compute time reaches the memory floor."""
+    return (params * bits_per_weight / 8 / bytes_per_s) / (2 * params / flops_per_s)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def replica_seed(base, rank):
+    """Each rank draws its own replica of the workload (weak scaling)."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload
+class DecodeStack:
+    """Quantized Llama-3-8B-shaped linears, LAYERS copies, plus per-GEMM activations/outputs."""
+
+    def __init__(self, torch, native, synthetic, seed, layers=LAYERS, M=1):
+        self.torch, self.native = torch, native
+        dev = torch.device("cuda")
+        self.M = M
+        self.layers = []
+        uniq = []
+        for i, (name, K, N) in enumerate(LLAMA8B_LINEARS):
+            Wb = synthetic.weights_normal(K, N, seed + i)
+            W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).to(dev)
+            codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
+            uniq.append((name, K, N, codes, scales, zeros))
+            del W
+        self.tiled = tiled_supported(torch, native, uniq[0][1:6])
+        for _ in range(layers):
+            lay = []
+            for (name, K, N, codes, scales, zeros) in uniq:
+                w = {"name": name, "K": K, "N": N, "weight_bytes": codes.numel() * 4 +
+                     scales.numel() * 2 + (0 if zeros is None else zeros.numel() * 4)}
+                if self.tiled:
+                    w["tiled"] = native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM)
+                else:
+                    w["codes"], w["scales"] = codes.clone(), scales.clone()
+                    w["zeros"] = None if zeros is None else zeros.clone()
+                lay.append(w)
+            self.layers.append(lay)
+        del uniq
+        # activations: one flat device buffer (and a pinned host twin for the e2e leg)
+        self.a_elems = sum(M * K for (_, K, _) in LLAMA8B_LINEARS) * layers
+        self.c_elems = sum(M * N for (_, _, N) in LLAMA8B_LINEARS) * layers
+        Ab = synthetic.activations(1, self.a_elems, seed + 100)
+        self.A_host = torch.from_numpy(Ab.view(np.int16)).view(torch.float16).pin_memory()
+        self.A = self.A_host.to(dev)
+        self.C = torch.empty(self.c_elems, dtype=torch.float16, device=dev)
+        self.C_host = torch.empty(self.c_elems, dtype=torch.float16).pin_memory()
+        ws = max(native.w4a16_workspace_bytes(M, N, K, GROUP) for (_, K, N) in LLAMA8B_LINEARS)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        # views per GEMM
+        self.calls = []
+        ao = co = 0
+        for lay in self.layers:
+            for w in lay:
+                K, N = w["K"], w["N"]
+                self.calls.append((w, self.A[ao:ao + M * K].view(M, K), self.C[co:co + M * N].view(M, N)))
+                ao += M * K
+                co += M * N
+        self.bytes_per_step = sum(algorithmic_bytes(M, w["K"], w["N"]) for (w, _, _) in self.calls)
+        self.weight_bytes = sum(w["weight_bytes"] for (w, _, _) in self.calls)
+
+    def gemm(self, w, A, C):
+        nat = self.native
+        if self.tiled:
+            nat.w4a16_gemm(A, w["tiled"], None, None, w["N"], GROUP, SYM, layout=nat.LAYOUT_TILED,
+                           C=C, workspace=self.ws)
+        else:
+            nat.w4a16_gemm(A, w["codes"], w["scales"], w["zeros"], w["N"], GROUP, SYM, C=C,
+                           workspace=self.ws)
+
+    def step(self):
+        for (w, A, C) in self.calls:
+            self.gemm(w, A, C)
+
+
+def tiled_supported(torch, native, qw):
+    """Whether the library runs the tiled layout (probed with one small call)."""
+    K, N, codes, scales, zeros = qw
+    try:
+        t = native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM)
+        A = torch.zeros((1, K), dtype=torch.float16, device=codes.device)
+        native.w4a16_gemm(A, t, None, None, N, GROUP, SYM, layout=native.LAYOUT_TILED)
+        torch.cuda.synchronize()
+        return True
+    except native.W4A16Error as e:
+        if e.status == native.EUNSUPPORTED:
+            return False
+        raise
+
+
+def count_graph_kernels(graph):
+    """Kernel nodes in a captured torch CUDA graph (None when the graph cannot be inspected)."""
+    try:
+        from cuda.bindings import runtime as cudart
+        raw = graph.raw_cuda_graph()
+        err, nodes, n = cudart.cudaGraphGetNodes(raw, 0)
+        err, nodes, n = cudart.cudaGraphGetNodes(raw, n)
+        count = 0
+        for node in nodes:
+            err, typ = cudart.cudaGraphNodeGetType(node)
+            if typ == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                count += 1
+        return count
+    except Exception:
+        return None
+
+
+def time_graph(torch, graph, steps, world, dev):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    return start.elapsed_time(end) / steps
+
+
+def time_per_launch(torch, stack, steps):
+    """Per-GEMM device durations (CUDA events on the launching stream) for `steps` steps.
+    A long sleep kernel first lets the host queue the launches ahead, so the events bracket
+    device execution only. Returns {shape name: [ms, ...]}."""
+    stream = torch.cuda.current_stream()
+    out = {}
+    for _ in range(steps):
+        evs = []
+        torch.cuda._sleep(int(60e6))
+        for (w, A, C) in stack.calls:
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            stack.gemm(w, A, C)
+            e.record(stream)
+            evs.append((w["name"], w["K"], w["N"], s, e))
+        torch.cuda.synchronize()
+        for (name, K, N, s, e) in evs:
+            out.setdefault((name, K, N), []).append(s.elapsed_time(e))
+    return out
+
+
+def time_e2e(torch, stack, steps, warmup):
+    """The step through the public Python API, inputs from pinned host memory, outputs read
+    back to pinned host memory every step; CUDA events around the whole step."""
+    for _ in range(warmup):
+        stack.A.copy_(stack.A_host, non_blocking=True)
+        stack.step()
+        stack.C_host.copy_(stack.C, non_blocking=True)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        stack.A.copy_(stack.A_host, non_blocking=True)
+        stack.step()
+        stack.C_host.copy_(stack.C, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
+    """TFLOPS of the (8192, 28672) sweep layer at M = 256, bf16 activations, rotating `copies`
+    distinct weight copies (122 MB each) so that L2 cannot serve repeats."""
+    dev = torch.device("cuda")
+    K, N, M = SWEEP_K, SWEEP_N, SWEEP_M
+    Wb = synthetic.weights_outliers(K, N, seed)
+    W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).to(dev)
+    codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
+    del W
+    use_tiled = tiled_supported(torch, native, (K, N, codes, scales, zeros))
+    ws_need = native.w4a16_workspace_bytes(M, N, K, GROUP)
+    ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+    if use_tiled:
+        mats = [(None, None, None, native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM))
+                for _ in range(copies)]
+    else:
+        mats = [(codes.clone(), scales.clone(), zeros.clone(), None) for _ in range(copies)]
+    del codes, scales, zeros
+    Ab = synthetic.activations(M, K, seed + 1, dtype=synthetic.BF16)
+    A = torch.from_numpy(Ab.view(np.int16)).view(torch.bfloat16).to(dev)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def run(i):
+        c, s, z, t = mats[i % copies]
+        if t is not None:
+            native.w4a16_gemm(A, t, None, None, N, GROUP, SYM, layout=native.LAYOUT_TILED, C=C,
+                              workspace=ws)
+        else:
+            native.w4a16_gemm(A, c, s, z, N, GROUP, SYM, C=C, workspace=ws)
+
+    for i in range(warmup):
+        run(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    durs = []
+    torch.cuda._sleep(int(20e6))
+    evs = []
+    for i in range(steps * copies):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        run(i)
+        e.record(stream)
+        evs.append((s, e))
+    torch.cuda.synchronize()
+    durs = [s.elapsed_time(e) for (s, e) in evs]
+    ms = statistics.mean(durs)
+    kernel = native.w4a16_select_kernel(M, N, K, GROUP)
+    return {"M": M, "K": K, "N": N, "ms": ms, "tflops": gemm_flops(M, K, N) / (ms * 1e-3) / 1e12,
+            "kernel": {1: "gemv", 2: "tc"}.get(kernel, str(kernel)), "dtype": "bf16",
+            "bytes": algorithmic_bytes(M, K, N), "launches": len(durs),
+            "layout": "tiled" if use_tiled else "plain"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(synthetic, seed, threads, budget_s=15.0, min_reps=1):
+    """The FP64 oracle's layer throughput on one Llama-3-8B layer (all four linears, all
+    columns, M = 1, fp16), repeated while under budget. Returns (GB/s, seconds, reps)."""
+    import oracle
+
+    packed = []
+    for i, (name, K, N) in enumerate(LLAMA8B_LINEARS):
+        Wb = synthetic.weights_normal(K, N, seed + i)
+        st, c, s, z = oracle.quantize(Wb, GROUP, SYM, nthreads=threads)
+        Ab = synthetic.activations(1, K, seed + 200 + i)
+        packed.append((K, N, c, s, z, Ab))
+    reps, total, nbytes = 0, 0.0, 0
+    while reps < min_reps or total < budget_s:
+        for (K, N, c, s, z, Ab) in packed:
+            t0 = time.perf_counter()
+            oracle.linear(Ab, 0, c, s, z, N, GROUP, SYM, nthreads=threads)
+            total += time.perf_counter() - t0
+            nbytes += algorithmic_bytes(1, K, N)
+        reps += 1
+        if total > budget_s:
+            break
+    return nbytes / total / 1e9, total, reps
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from weight_only_int4_07_b200 import synthetic
+
+    threads = host_cores()
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample(synthetic, 11, threads, budget_s=0.0)
+    for _ in range(args.steps):
+        gbs, secs, reps = oracle_sample(synthetic, 11, threads, budget_s=0.0)
+        per_step.append((gbs, secs))
+    value = statistics.mean(g for g, _ in per_step)
+    ms = 1e3 * statistics.mean(s for _, s in per_step)
+    sample = ("one Llama-3-8B-shaped layer per step: the four decode linears (4096x6144, 4096x4096, "
+              "4096x28672, 14336x4096), all columns, M=1, g128 asym, fp16; FP64 oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama3-8b decode linears, M=1, g128 asym INT4, fp16 acts",
+                       "layers_per_step": 1},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    from weight_only_int4_07_b200 import build, native, synthetic
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    native.lib()
+    peaks = load_peaks()
+
+    seed = replica_seed(1000, rank)
+    stack = DecodeStack(torch, native, synthetic, seed)
+    torch.cuda.synchronize()
+
+    # warm-up, then capture one step in a CUDA graph
+    for _ in range(max(args.warmup, 1)):
+        stack.step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        stack.step()
+    torch.cuda.synchronize()
+    kernels_per_step = count_graph_kernels(graph)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    with ClockSampler(local_rank) as clk:
+        ms = time_graph(torch, graph, args.steps, world, dev)
+    ms_max = max_over_ranks(ms, world, dev)
+    value = world * stack.bytes_per_step / (ms_max * 1e-3) / 1e9
+
+    # per-launch device durations (roofline of the dominant kernel)
+    launches = time_per_launch(torch, stack, max(1, min(args.steps, 5)))
+    tot_bytes = sum(algorithmic_bytes(1, K, N) * len(v) for (name, K, N), v in launches.items())
+    tot_ms = sum(sum(v) for v in launches.values())
+    n_launch = sum(len(v) for v in launches.values())
+    per_shape = {name: {"K": K, "N": N, "mean_us": 1e3 * statistics.mean(v),
+                        "gbs": algorithmic_bytes(1, K, N) / (statistics.mean(v) * 1e-3) / 1e9}
+                 for (name, K, N), v in launches.items()}
+    achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+    kernel = native.w4a16_select_kernel(1, 4096, 4096, GROUP)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": {1: "gemv", 2: "tc"}.get(kernel, str(kernel)),
+                "bytes_per_launch": tot_bytes / n_launch, "launch_us": 1e3 * tot_ms / n_launch,
+                "peak_source": peaks["source"], "per_shape": per_shape}
+
+    # end to end through the Python API, pinned host <-> device copies inside the timed region
+    e2e_ms = time_e2e(torch, stack, args.steps, args.warmup)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e = {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": stack.A.numel() * 2, "d2h_bytes_per_step": stack.C.numel() * 2,
+           "ms_per_step": e2e_ms}
+
+    del graph
+    torch.cuda.synchronize()
+    gemms_per_step = len(stack.calls)
+    layout = "tiled" if stack.tiled else "plain"
+    weight_bytes = stack.weight_bytes
+    bytes_per_step = stack.bytes_per_step
+
+    # M = 256 on the sweep layer (TFLOPS)
+    m256 = None
+    if not args.skip_m256:
+        del stack
+        torch.cuda.empty_cache()
+        r = bench_m256(torch, native, synthetic, replica_seed(5000, rank), max(2, min(args.steps, 10)),
+                       args.warmup)
+        ms256 = max_over_ranks(r["ms"], world, dev)
+        tf = gemm_flops(r["M"], r["K"], r["N"]) / (ms256 * 1e-3) / 1e12
+        peak_tf = peaks["bf16_tflops"]
+        m256 = {"value": world * tf, "unit": "TFLOP/s", "ms": ms256, "kernel": r["kernel"],
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": tf / peak_tf, "traffic": None, "peak_source": peaks["source"] +
+                             " burst"},
+                "config": {"M": r["M"], "K": r["K"], "N": r["N"], "group": GROUP, "sym": False,
+                           "acts": "bf16", "weights": "N(0,0.02) with 0.1% outliers x20",
+                           "l2": "4 rotating weight copies of 122 MB"}}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        threads = host_cores()
+        gbs, secs, reps = oracle_sample(synthetic, 11, threads, budget_s=args.cpu_budget)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{reps} pass(es) over one Llama-3-8B-shaped layer (4 decode linears, all "
+                         f"columns, M=1, g128 asym, fp16), FP64 oracle, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+                "data": "synthetic (seeded; weights N(0,0.02) fp16, activations N(0,1) fp16)",
+                "config": {"workload": "llama3-8b decode linears (qkv 4096x6144, o 4096x4096, "
+                                       "gate+up 4096x28672, down 14336x4096), M=1, g128 asym INT4, "
+                                       "fp16 acts, 32 layers per step",
+                           "layers": LAYERS, "gemms_per_step": gemms_per_step,
+                           "weight_bytes_per_step": weight_bytes,
+                           "algorithmic_bytes_per_step": bytes_per_step,
+                           "parallelism": f"replica x{world}", "layout": layout,
+                           "l2": "inputs larger than L2: 3.63 GB of packed weights per step",
+                           "timing": "CUDA graph replay of one step, CUDA events"},
+                "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
+                "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
+                "m256": m256}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--skip-m256", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,190 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) W4A16 weight-only INT4 linear layer.
+ *
+ * The layer: 16-bit activations A [M, K] times a weight matrix W [K, N] that is stored as 4-bit
+ * codes, eight per 32-bit word, with one FP16 scale per group of `group` consecutive input
+ * channels and, for the asymmetric scheme, one 4-bit zero-point per group. The kernel reads the
+ * codes, dequantizes them on chip, w = (q - z) * s, and multiplies them against the 16-bit
+ * activations with FP32 accumulation.
+ *   - "4.3 Weight-only INT4", section 1 "W4A16 storage and compute": eight 4-bit codes per
+ *     32-bit word, one FP16 scale per group, a zero-point for asymmetric schemes, dequantized
+ *     on chip to FP16/BF16, then multiplied with 16-bit activations.
+ *   - "INT4 and Low-Bit Inference -- Inference Optimization", section 6-9, "the packed layout":
+ *     qweight (K/8, N) int32, scales (K/g, N) fp16, qzeros (K/g, N/8) int32.
+ *   - "INT4 LLMs: What 4-Bit Quantization Means and When to Use It", section "What INT4 means in
+ *     an LLM": signed codes -8..7, two per byte.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers named as device buffers are CUDA device (or managed) memory of the current
+ *     device. The caller allocates and frees every buffer; the library never allocates memory and
+ *     never synchronises the device. Every call is asynchronous on `stream` (a cudaStream_t passed
+ *     as void*, NULL = the legacy default stream).
+ *   - Shapes: K % 8 == 0, N % 8 == 0, group in {32, 64, 128}, K % group == 0, M >= 1.
+ *     N % 8 == 0 also makes every row of A, C and the packed arrays 16-byte aligned when the
+ *     base pointers are (N = 8 with 16-bit C rows is 16 bytes).
+ *   - Device pointers must be 16-byte aligned.
+ *   - Arguments are checked on the host before any launch. A rejected call returns a negative
+ *     w4a16_status and launches nothing. A failed launch returns W4A16_ECUDA.
+ *   - Conditions found on the device are written to an optional device int `dev_status`
+ *     (first error wins; the caller zeroes it). They never fault or trap the GPU.
+ *   - The entry points are stateless and thread-safe, except where an entry point says otherwise.
+ *
+ * Packed layout ("plain", the checkpoint layout)
+ *   codes  int32 [K/8, N]   word (j, n), bits [4i, 4i+4): code of (k = 8j + i, n).
+ *                           symmetric: two's-complement nibble, value -8..7.
+ *                           asymmetric: unsigned nibble, value 0..15.
+ *   scales fp16  [K/g, N]   scale of group (g, n).
+ *   zeros  int32 [K/g, N/8] asymmetric only: word (g, j), bits [4i, 4i+4): zero of (g, n = 8j + i),
+ *                           unsigned 0..15. NULL for the symmetric scheme.
+ *   Dequantized weight: w[k, n] = (q[k, n] - z[k/g, n]) * s[k/g, n]  (z = 0 when symmetric).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Symbols of this header are the only ones the shared library exports. */
+#ifndef W4A16_API
+#define W4A16_API __attribute__((visibility("default")))
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. Zero is success; every error is negative. */
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_EINVAL = -1,        /* bad shape, null pointer, or a value outside its enum        */
+    W4A16_EALIGN = -2,        /* a device pointer is not 16-byte aligned                      */
+    W4A16_EUNSUPPORTED = -3,  /* a group size, dtype, layout or kernel choice not supported   */
+    W4A16_ENONFINITE = -4,    /* device: a weight group held Inf or NaN (via dev_status)      */
+    W4A16_EWORKSPACE = -5,    /* workspace smaller than w4a16_workspace_bytes()               */
+    W4A16_ECUDA = -6,         /* a CUDA runtime call or a kernel launch failed                */
+    W4A16_ETIMEOUT = -7       /* device: a bounded wait gave up (via dev_status)              */
+} w4a16_status;
+
+/* 16-bit activation (and output) type. */
+typedef enum { W4A16_F16 = 0, W4A16_BF16 = 1 } w4a16_dtype;
+
+/* Weight layout handed to w4a16_gemm. */
+typedef enum {
+    W4A16_LAYOUT_PLAIN = 0,   /* codes / scales / zeros as above                              */
+    W4A16_LAYOUT_TILED = 1    /* the single buffer written by w4a16_repack                    */
+} w4a16_layout;
+
+/* Kernel family chosen by the M-based dispatch (see w4a16_select_kernel). */
+typedef enum {
+    W4A16_KERNEL_AUTO = 0,    /* let the dispatch decide                                      */
+    W4A16_KERNEL_GEMV = 1,    /* split-K CUDA-core GEMV / skinny GEMM, M <= 16                */
+    W4A16_KERNEL_TC = 2       /* tcgen05 tensor-core GEMM with TMEM accumulators              */
+} w4a16_kernel;
+
+/*
+ * w4a16_quantize -- round-to-nearest group quantization of an FP16 weight matrix.
+ *   "INT4 LLMs: What 4-Bit Quantization Means and When to Use It", sections "What INT4 means in
+ *   an LLM" and "Why mapping to 16 values still works" (16 levels, group-wise scales, symmetric
+ *   grid centred on zero vs. affine grid with an offset); "4.3 Weight-only INT4", section 1.
+ *   For each group (g, n) of `group` consecutive k in column n, in FP64:
+ *     sym:  s = fp16(amax / 7),                              q = clamp(rne(w / s), -8, 7)
+ *     asym: lo = min(0, min w), hi = max(0, max w), s = fp16((hi - lo) / 15),
+ *           z = clamp(rne(-lo / s), 0, 15),                  q = clamp(rne(w / s) + z, 0, 15)
+ *   rne = round half to even; every division is an IEEE FP64 division. A group whose scale rounds
+ *   to zero stores s = 1, z = 0 and q = z.
+ * Arguments
+ *   W          device, fp16 [K, N] row-major (n fastest).
+ *   K, N       input channels (rows of W) and output channels (columns).
+ *   group      32, 64 or 128.
+ *   sym        1 = symmetric (no zeros), 0 = asymmetric.
+ *   codes      device out, int32 [K/8, N].
+ *   scales     device out, fp16 [K/g, N].
+ *   zeros      device out, int32 [K/g, N/8] when sym == 0; must be NULL when sym == 1.
+ *   dev_status device int or NULL. Set to W4A16_ENONFINITE when a group holds Inf/NaN (that
+ *              group's outputs are then unspecified).
+ *   stream     cudaStream_t.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED or W4A16_ECUDA.
+ */
+W4A16_API int w4a16_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes, void* scales,
+                   int32_t* zeros, int* dev_status, void* stream);
+
+/*
+ * w4a16_repack_bytes -- size in bytes of the tiled buffer for a K x N weight (0 on bad shape).
+ */
+W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);
+
+/*
+ * w4a16_repack -- one-time load-time permutation of the plain packed layout into the tiled
+ * layout that w4a16_gemm reads fastest. It is a bijection of bits: nothing is rounded or
+ * re-quantized. "INT4 and Low-Bit Inference", section 5 "The kernel is half the story" (weights
+ * pre-permuted at load so unpacking is branch-free and coalesced); "4.3 Weight-only INT4",
+ * section 4 (weights pre-reordered into a layout that suits runtime reads).
+ * Tiled layout: the weight is cut into tiles of 128 output channels x 64 input channels
+ * (tile (t, c) covers n in [128 t, 128 t + 128), k in [64 c, 64 c + 64)). Tiles are stored in
+ * order c-major-within-t: tile index = t * (K / 64) + c; each tile is 128 x 8 = 1024 int32 words
+ * (4 KiB) holding word (j, n) of the plain layout at offset
+ *     ((j % 8) / 4) * 512 + (n % 128) * 4 + (j % 4)            (j = 8 c + j % 8)
+ * so that one 16-byte vector holds four consecutive words along K of one output channel, and a
+ * warp's 32 consecutive output channels read 512 contiguous bytes. Scales and zeros follow the
+ * codes in the same buffer, in the plain layouts [K/g, N] fp16 and [K/g, N/8] int32 (asym),
+ * each starting on a 256-byte boundary.
+ * Requires N % 128 == 0 and K % 64 == 0 (else W4A16_EUNSUPPORTED).
+ * Arguments: codes, scales, zeros as produced by w4a16_quantize (zeros NULL iff sym);
+ * tiled = device out of w4a16_repack_bytes() bytes; stream.
+ */
+W4A16_API int w4a16_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
+                 int group, int sym, void* tiled, void* stream);
+
+/*
+ * w4a16_workspace_bytes -- device scratch that w4a16_gemm needs for an M x N x K call with the
+ * kernel the dispatch picks (split-K partial sums and their counters). 0 when none is needed.
+ */
+W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
+
+/*
+ * w4a16_select_kernel -- the M-based dispatch, as a pure host function: returns the
+ * w4a16_kernel that w4a16_gemm(..., W4A16_KERNEL_AUTO) runs for this shape. Small M is bound
+ * by the weight stream and goes to the split-K GEMV; larger M goes to the tensor-core GEMM
+ * ("INT8 vs INT4 Quantization, in depth", section "Two regimes: waiting for memory, waiting
+ * for math"). The environment variable W4A16_FORCE_KERNEL=gemv|tc overrides the choice.
+ */
+W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
+
+/*
+ * w4a16_gemm -- C[M, N] = A[M, K] . dequant(W)[K, N], FP32 accumulation, C in the dtype of A.
+ *   "4.3 Weight-only INT4", section 4 (read, unpack, dequantize and multiply in one kernel, so
+ *   each weight byte crosses HBM once); section 1 (dequantize on chip, 16-bit multiply inputs).
+ * Arguments
+ *   A          device, [M, K] row-major, fp16 or bf16 (a_dtype).
+ *   a_dtype    W4A16_F16 or W4A16_BF16. C has the same type.
+ *   M, K       rows of A; input channels.
+ *   wq         device: codes int32 [K/8, N] (layout PLAIN) or the w4a16_repack buffer (TILED).
+ *   layout     W4A16_LAYOUT_PLAIN or W4A16_LAYOUT_TILED.
+ *   scales     device fp16 [K/g, N] for PLAIN; ignored (may be NULL) for TILED.
+ *   zeros      device int32 [K/g, N/8] for PLAIN asymmetric; NULL for symmetric; ignored for TILED.
+ *   N, group   output channels; group size.
+ *   sym        1 = symmetric codes, 0 = asymmetric (must match how the weight was quantized).
+ *   C          device out, [M, N] row-major, dtype a_dtype. Must not alias A or the weights.
+ *   workspace  device scratch of at least w4a16_workspace_bytes(M, N, K, group) bytes (NULL if 0).
+ *              Calls that share one workspace must be ordered on the GPU (same stream).
+ *   ws_bytes   size of workspace.
+ *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC.
+ *   stream     cudaStream_t.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
+ * W4A16_ECUDA.
+ */
+W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* wq, int layout,
+               const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
+               void* workspace, size_t ws_bytes, int kernel, void* stream);
+
+/* w4a16_status_str -- a static, human-readable name for a status code. */
+W4A16_API const char* w4a16_status_str(int status);
+
+/* w4a16_version -- library version as 10000 * major + 100 * minor + patch. */
+W4A16_API int w4a16_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

@@ -9,7 +9,7 @@ import os
 
 import numpy as np
 
-from .build import build
+from .build import build as _build
 
 F16 = 0
 BF16 = 1
@@ -23,7 +23,7 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        path = build()
+        path = _build()
         lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         L = ctypes.c_long
@@ -54,6 +54,10 @@ def _load():
         lib.w4o_linear.restype = I
         lib.w4o_matmul.argtypes = [P, I, L, L, P, L, P]
         lib.w4o_matmul.restype = None
+        lib.w4o_tiled_offsets.argtypes = [L, L, L, I, P]
+        lib.w4o_tiled_offsets.restype = None
+        lib.w4o_repack.argtypes = [P, P, P, L, L, L, I, P]
+        lib.w4o_repack.restype = I
         lib.w4o_max_threads.argtypes = []
         lib.w4o_max_threads.restype = I
         _lib = lib
@@ -178,3 +182,25 @@ def within_bound(y, y_ref, y_abs, rel=2e-3, abs_=1e-5):
     """The acceptance bound |y - y_ref| <= rel * sum_k |a_k w_k| + abs_, elementwise."""
     y = np.asarray(y, dtype=np.float64)
     return np.abs(y - y_ref) <= rel * y_abs + abs_
+
+
+# ----------------------------------------------------------------------------- tiled layout
+def tiled_offsets(K, N, group, sym):
+    """dict of byte offsets/sizes of the tiled buffer's regions and its total size."""
+    out = np.zeros(7, dtype=np.int64)
+    _load().w4o_tiled_offsets(K, N, group, int(sym), _ptr(out))
+    keys = ("codes", "codes_bytes", "scales", "scales_bytes", "zeros", "zeros_bytes", "total")
+    return {k: int(v) for k, v in zip(keys, out)}
+
+
+def repack(codes, scales, zeros, K, N, group, sym):
+    """The tiled buffer (uint8) holding the same bits as the plain packed weight."""
+    off = tiled_offsets(K, N, group, sym)
+    out = np.zeros(off["total"], dtype=np.uint8)
+    c = _c(codes, np.int32)
+    s = _c(scales, np.uint16)
+    z = None if sym else _c(zeros, np.int32)
+    st = _load().w4o_repack(_ptr(c), _ptr(s), _ptr(z), K, N, group, int(sym), _ptr(out))
+    if st != OK:
+        raise ValueError(f"oracle repack rejected its arguments (status {st})")
+    return out

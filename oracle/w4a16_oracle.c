@@ -323,3 +323,51 @@ int w4o_max_threads(void) {
     return 1;
 #endif
 }
+
+/* ---------------------------------------------------------------------------------------------
+ * The tiled weight buffer of the library's repack entry point, restated from its definition:
+ * tiles of 128 output channels x 64 input channels (8 packed rows); tile (t, c) has index
+ * t * (K/64) + c and holds 1024 words; plain word (j, n) sits at
+ *   ((j mod 8) div 4) * 512 + (n mod 128) * 4 + (j mod 4)
+ * inside its tile. Scales (plain [K/g, N] fp16) and zeros (plain [K/g, N/8] int32, asym only)
+ * follow, each region starting at a multiple of 256 bytes. Padding bytes are left zero.
+ * (The pages ask for a pre-permuted layout -- "INT4 and Low-Bit Inference", section 5
+ * "The kernel is half the story" -- but leave its form open; this one is the library's.)
+ * ------------------------------------------------------------------------------------------- */
+static long round_up_256(long x) { return (x + 255) / 256 * 256; }
+
+void w4o_tiled_offsets(long K, long N, long group, int sym, long* out) {
+    const long codes_bytes = K * N / 2;
+    const long scales_off = round_up_256(codes_bytes);
+    const long scales_bytes = (K / group) * N * 2;
+    const long zeros_off = round_up_256(scales_off + scales_bytes);
+    const long zeros_bytes = sym ? 0 : (K / group) * (N / 8) * 4;
+    out[0] = 0;
+    out[1] = codes_bytes;
+    out[2] = scales_off;
+    out[3] = scales_bytes;
+    out[4] = zeros_off;
+    out[5] = zeros_bytes;
+    out[6] = round_up_256(zeros_off + zeros_bytes);
+}
+
+int w4o_repack(const int32_t* codes, const uint16_t* scales, const int32_t* zeros, long K, long N,
+               long group, int sym, uint8_t* out) {
+    if (!valid_shape(K, N, group) || N % 128 != 0 || K % 64 != 0) return W4O_EINVAL;
+    long off[7];
+    w4o_tiled_offsets(K, N, group, sym, off);
+    memset(out, 0, (size_t)off[6]);
+    int32_t* tiled = (int32_t*)out;
+    const long ktiles = K / 64;
+    for (long t = 0; t < N / 128; ++t)
+        for (long c = 0; c < ktiles; ++c)
+            for (long jl = 0; jl < 8; ++jl)
+                for (long nl = 0; nl < 128; ++nl) {
+                    const long j = 8 * c + jl, n = 128 * t + nl;
+                    const long pos = (t * ktiles + c) * 1024 + (jl / 4) * 512 + nl * 4 + (jl % 4);
+                    tiled[pos] = codes[j * N + n];
+                }
+    memcpy(out + off[2], scales, (size_t)off[3]);
+    if (!sym) memcpy(out + off[4], zeros, (size_t)off[5]);
+    return W4O_OK;
+}

@@ -1,0 +1,146 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the headers declare,
+and its host-side logic (argument checks, sizes, dispatch) answers without touching a device.
+
+Every call below either is a pure host function or is rejected by the host-side checks before
+any CUDA call is made; no compute call is issued.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from weight_only_int4_07_b200 import native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*W4A16_API\s+[\w\s\*]+?\b(w4a16_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from weight_only_int4_07_b200 import build
+
+    build.build()
+    return native.lib()
+
+
+def test_headers_declare_the_entry_points():
+    names = _declared_symbols()
+    for required in ("w4a16_quantize", "w4a16_gemm", "w4a16_repack", "w4a16_repack_bytes",
+                     "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+        assert getattr(L, name) is not None
+
+
+def test_library_exports_nothing_else(L):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", native.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert exported == set(_declared_symbols())
+
+
+def test_status_strings(L):
+    assert native.status_str(0) == "W4A16_OK"
+    assert native.status_str(-5) == "W4A16_EWORKSPACE"
+    assert native.status_str(12345) == "W4A16_UNKNOWN"
+    assert native.w4a16_version() >= 100
+
+
+def test_repack_bytes(L):
+    # codes K*N/2, then scales (K/g)*N*2 and zeros (K/g)*(N/8)*4, each on a 256-byte boundary
+    K, N, g = 4096, 4096, 128
+    codes = K * N // 2
+    scales = (K // g) * N * 2
+    zeros = (K // g) * (N // 8) * 4
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert native.w4a16_repack_bytes(K, N, g, 0) == up(up(up(codes) + scales) + zeros)
+    assert native.w4a16_repack_bytes(K, N, g, 1) == up(up(codes) + scales)
+    assert native.w4a16_repack_bytes(K, 8, g, 0) == 0          # N not a multiple of 128
+    assert native.w4a16_repack_bytes(96, 128, 32, 0) == 0      # K not a multiple of 64
+    assert native.w4a16_repack_bytes(4096, 4096, 48, 0) == 0   # group not supported
+
+
+def test_select_kernel_and_workspace_are_host_only(L):
+    for M in (1, 2, 16, 17, 32, 256, 2048):
+        k = native.w4a16_select_kernel(M, 4096, 4096, 128)
+        assert k in (native.KERNEL_GEMV, native.KERNEL_TC)
+        assert native.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
+    assert native.w4a16_workspace_bytes(0, 4096, 4096, 128) == 0
+    assert native.w4a16_workspace_bytes(1, 4096, 4000, 128) == 0
+
+
+# Fake device addresses: the checks below reject the call before any CUDA call, so the
+# addresses are never dereferenced.
+A16 = ctypes.c_void_p(1 << 20)
+B16 = ctypes.c_void_p(2 << 20)
+C16 = ctypes.c_void_p(3 << 20)
+D16 = ctypes.c_void_p(4 << 20)
+MIS = ctypes.c_void_p((5 << 20) + 8)
+
+
+def _gemm(L, A=A16, dt=0, M=1, K=256, wq=B16, layout=0, scales=C16, zeros=D16, N=256, g=128,
+          sym=0, C=A16, ws=None, wsb=1 << 30, kernel=0):
+    return L.w4a16_gemm(A, dt, M, K, wq, layout, scales, zeros, N, g, sym, C, ws, wsb, kernel, None)
+
+
+def test_gemm_rejects_bad_arguments(L):
+    assert _gemm(L, K=100) == native.EINVAL                    # K % 8
+    assert _gemm(L, N=100) == native.EINVAL                    # N % 8
+    assert _gemm(L, K=264, g=128) == native.EINVAL             # K % group
+    assert _gemm(L, g=16) == native.EUNSUPPORTED               # group
+    assert _gemm(L, M=0) == native.EINVAL
+    assert _gemm(L, dt=2) == native.EINVAL
+    assert _gemm(L, layout=3) == native.EINVAL
+    assert _gemm(L, sym=2) == native.EINVAL
+    assert _gemm(L, kernel=7) == native.EINVAL
+    assert _gemm(L, A=None) == native.EINVAL
+    assert _gemm(L, wq=None) == native.EINVAL
+    assert _gemm(L, C=None) == native.EINVAL
+    assert _gemm(L, scales=None) == native.EINVAL
+    assert _gemm(L, zeros=None, sym=0) == native.EINVAL        # asymmetric needs zeros
+    assert _gemm(L, zeros=D16, sym=1) == native.EINVAL         # symmetric takes none
+    assert _gemm(L, A=MIS) == native.EALIGN
+    assert _gemm(L, C=MIS) == native.EALIGN
+    assert _gemm(L, scales=MIS) == native.EALIGN
+    assert _gemm(L, layout=1, N=8) == native.EUNSUPPORTED      # tiled needs N % 128
+    need = native.w4a16_workspace_bytes(1, 256, 256, 128)
+    if need > 0:
+        assert _gemm(L, ws=D16, wsb=need - 1) == native.EWORKSPACE
+        assert _gemm(L, ws=None, wsb=need) == native.EWORKSPACE
+        assert _gemm(L, ws=MIS, wsb=need) == native.EALIGN
+
+
+def test_quantize_rejects_bad_arguments(L):
+    q = L.w4a16_quantize
+    assert q(A16, 256, 256, 128, 0, B16, C16, None, None, None) == native.EINVAL   # asym, no zeros
+    assert q(A16, 256, 256, 128, 1, B16, C16, D16, None, None) == native.EINVAL    # sym, zeros
+    assert q(A16, 250, 256, 128, 0, B16, C16, D16, None, None) == native.EINVAL
+    assert q(A16, 256, 256, 100, 0, B16, C16, D16, None, None) == native.EUNSUPPORTED
+    assert q(MIS, 256, 256, 128, 0, B16, C16, D16, None, None) == native.EALIGN
+    assert q(None, 256, 256, 128, 0, B16, C16, D16, None, None) == native.EINVAL
+    assert q(A16, 256, 256, 128, 3, B16, C16, D16, None, None) == native.EINVAL
+
+
+def test_repack_rejects_bad_arguments(L):
+    r = L.w4a16_repack
+    assert r(A16, B16, C16, 256, 8, 128, 0, D16, None) == native.EUNSUPPORTED
+    assert r(A16, B16, None, 256, 128, 128, 0, D16, None) == native.EINVAL
+    assert r(A16, B16, C16, 256, 128, 128, 1, D16, None) == native.EINVAL
+    assert r(A16, B16, C16, 256, 128, 128, 0, MIS, None) == native.EALIGN

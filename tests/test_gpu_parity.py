@@ -1,0 +1,254 @@
+"""GPU parity: the CUDA path against the FP64 oracle, element by element, through the C ABI.
+
+Bars: codes, scales, zeros and the repacked buffer bit-exact; every GEMM output within
+|y - y_ref| <= 2e-3 * sum_k |a_k * w_k| + 1e-5, y the kernel's 16-bit output widened to FP64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_int4_07_b200 import native, synthetic
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+_cache = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from weight_only_int4_07_b200 import build
+
+    build.build()
+    native.lib()
+    torch.cuda.set_device(0)
+
+
+def _weights(kind, K, N, seed):
+    key = ("W", kind, K, N, seed)
+    if key not in _cache:
+        gen = {"normal": synthetic.weights_normal, "outliers": synthetic.weights_outliers,
+               "student_t": synthetic.weights_student_t}[kind]
+        _cache[key] = gen(K, N, seed)
+    return _cache[key]
+
+
+def _quantized(kind, K, N, group, sym, seed):
+    """(W bits, oracle codes/scales/zeros, GPU codes/scales/zeros)."""
+    key = ("Q", kind, K, N, group, sym, seed)
+    if key not in _cache:
+        Wb = _weights(kind, K, N, seed)
+        st, oc, os_, oz = oracle.quantize(Wb, group, sym)
+        assert st == oracle.OK
+        W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
+        gc, gs, gz = native.w4a16_quantize(W, group, sym)
+        torch.cuda.synchronize()
+        _cache[key] = (Wb, (oc, os_, oz), (gc, gs, gz))
+    return _cache[key]
+
+
+def _to_np16(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _acts(M, K, seed, dtype):
+    Ab = synthetic.activations(M, K, seed, dtype=dtype)
+    tdt = torch.float16 if dtype == synthetic.F16 else torch.bfloat16
+    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+    return Ab, A
+
+
+def _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=None):
+    Y, Yabs = oracle.linear(Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    y = oracle.decode16(_to_np16(C), a_dtype)
+    if cols is not None:
+        y = y[:, cols]
+    err = np.abs(y - Y)
+    bound = REL * Yabs + ABS
+    bad = err > bound
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outputs outside the bound; worst ratio "
+                           f"{(err / bound).max():.3f}")
+    return float((err / bound).max())
+
+
+# ----------------------------------------------------------------------------- quantize
+QUANT_CASES = [
+    # kind, K, N, group, sym, seed
+    ("normal", 512, 256, 128, 0, 0),          # the tiny configuration
+    ("normal", 384, 264, 32, 1, 1),           # ragged N (not a multiple of the 256-thread block)
+    ("student_t", 1024, 520, 64, 0, 2),
+    ("outliers", 2048, 1032, 128, 1, 3),
+    ("normal", 4096, 6144, 128, 0, 4),        # 8B qkv shape
+    ("student_t", 8192, 8192, 32, 1, 5),      # format variant, full size
+    ("outliers", 8192, 28672, 128, 0, 6),     # sweep shape, full size
+]
+
+
+@pytest.mark.parametrize("kind,K,N,group,sym,seed", QUANT_CASES)
+def test_quantize_bit_exact(kind, K, N, group, sym, seed):
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized(kind, K, N, group, sym, seed)
+    assert np.array_equal(gc.cpu().numpy(), oc)
+    assert np.array_equal(_to_np16(gs), os_)
+    if sym:
+        assert gz is None
+    else:
+        assert np.array_equal(gz.cpu().numpy(), oz)
+
+
+def test_quantize_degenerate_groups_bit_exact():
+    K, N, group = 256, 128, 32
+    Wb = synthetic.weights_normal(K, N, seed=7).copy()
+    Wb[:32, 5] = 0                     # all-zero group
+    Wb[32:64, 9] = 0x0001              # sub-2^-25 range: scale rounds to zero
+    for sym in (0, 1):
+        st, oc, os_, oz = oracle.quantize(Wb, group, sym)
+        W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
+        gc, gs, gz = native.w4a16_quantize(W, group, sym)
+        assert np.array_equal(gc.cpu().numpy(), oc)
+        assert np.array_equal(_to_np16(gs), os_)
+        if not sym:
+            assert np.array_equal(gz.cpu().numpy(), oz)
+
+
+def test_quantize_reports_nonfinite():
+    K, N, group = 256, 128, 128
+    Wb = synthetic.weights_normal(K, N, seed=8).copy()
+    Wb[77, 3] = 0x7C00                 # +inf
+    for sym in (0, 1):
+        W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        gc, gs, gz = native.w4a16_quantize(W, group, sym, dev_status=status)
+        assert int(status.item()) == native.ENONFINITE
+        # the other groups are still exact
+        st, oc, os_, oz = oracle.quantize(Wb, group, sym)
+        assert st == oracle.ENONFINITE
+        ok_cols = np.arange(N) != 3
+        assert np.array_equal(gc.cpu().numpy()[:, ok_cols], oc[:, ok_cols])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    W = torch.from_numpy(synthetic.weights_normal(K, N, seed=9).view(np.int16)).view(torch.float16).cuda()
+    native.w4a16_quantize(W, group, 0, dev_status=status)
+    assert int(status.item()) == 0
+
+
+# ----------------------------------------------------------------------------- repack
+@pytest.mark.parametrize("K,N,group,sym", [(512, 256, 128, 0), (256, 384, 32, 1), (4096, 6144, 128, 0),
+                                            (8192, 8192, 32, 1)])
+def test_repack_bit_exact(K, N, group, sym):
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("normal" if K < 8192 else "student_t", K, N, group,
+                                                 sym, 4 if K == 4096 else (5 if K == 8192 else 11))
+    ref = oracle.repack(oc, os_, oz, K, N, group, sym)
+    off = oracle.tiled_offsets(K, N, group, sym)
+    assert native.w4a16_repack_bytes(K, N, group, sym) == off["total"]
+    buf = native.w4a16_repack(gc, gs, gz, K, N, group, sym).cpu().numpy()
+    for region in ("codes", "scales", "zeros"):
+        a, n = off[region], off[region + "_bytes"]
+        assert np.array_equal(buf[a:a + n], ref[a:a + n]), region
+
+
+# ----------------------------------------------------------------------------- GEMM, small
+SMALL_GEMM = [
+    # M, K, N, group, sym, a_dtype
+    (1, 512, 256, 128, 0, 0),     # the tiny configuration
+    (1, 384, 264, 32, 1, 1),
+    (2, 1024, 520, 64, 0, 0),
+    (3, 256, 1032, 128, 1, 1),
+    (5, 768, 136, 32, 0, 1),
+    (8, 1024, 264, 128, 0, 0),
+    (13, 512, 392, 64, 1, 0),
+    (16, 2048, 1032, 128, 0, 1),
+    (17, 512, 256, 32, 0, 0),
+    (33, 1024, 520, 128, 1, 1),
+    (64, 512, 384, 64, 0, 0),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SMALL_GEMM)
+@pytest.mark.parametrize("kernel", [native.KERNEL_AUTO, native.KERNEL_GEMV])
+def test_gemm_small_full_output(M, K, N, group, sym, a_dtype, kernel):
+    kind = "student_t" if sym else "normal"
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized(kind, K, N, group, sym, 20 + K + N)
+    Ab, A = _acts(M, K, 100 + M, a_dtype)
+    C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym, kernel=kernel)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+@pytest.mark.parametrize("sym", [0, 1])
+def test_gemm_unit_rows_return_dequantized_rows(a_dtype, sym):
+    K, N, group = 512, 256, 64
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("normal", K, N, group, sym, 31)
+    rows = [0, 1, 7, 8, 63, 64, 200, 511]
+    Ab = np.zeros((len(rows), K), dtype=np.uint16)
+    one = 0x3C00 if a_dtype == 0 else 0x3F80
+    for i, k in enumerate(rows):
+        Ab[i, k] = one
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+    C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
+    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
+    expect = oracle.decode16(oracle.encode16(What[rows], a_dtype), a_dtype)   # one rounding
+    got = oracle.decode16(_to_np16(C), a_dtype)
+    assert np.array_equal(got, expect)
+
+
+def test_gemm_zero_weights_give_zero():
+    K, N, group = 256, 128, 32
+    Wb = np.zeros((K, N), dtype=np.uint16)
+    W = torch.zeros((K, N), dtype=torch.float16, device="cuda")
+    for sym in (0, 1):
+        gc, gs, gz = native.w4a16_quantize(W, group, sym)
+        Ab, A = _acts(4, K, 5, 0)
+        C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
+        assert torch.count_nonzero(C).item() == 0
+    assert Wb.sum() == 0
+
+
+def test_gemm_deterministic():
+    M, K, N, group = 4, 2048, 1032, 128
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("normal", K, N, group, 0, 40)
+    Ab, A = _acts(M, K, 41, 1)
+    C1 = native.w4a16_gemm(A, gc, gs, gz, N, group, 0)
+    C2 = native.w4a16_gemm(A, gc, gs, gz, N, group, 0)
+    assert torch.equal(C1.view(torch.int16), C2.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- full-size, sampled
+LLAMA8B = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)]
+
+
+@pytest.mark.parametrize("K,N", LLAMA8B)
+def test_gemm_llama8b_decode_sampled(K, N):
+    group, sym, a_dtype = 128, 0, 0
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("normal", K, N, group, sym, 1000 + N)
+    Ab, A = _acts(1, K, 2000 + K, a_dtype)
+    cols = synthetic.column_sample(N, 512, seed=K + N)
+    C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("M", [1, 16, 256])
+def test_gemm_sweep_shape_sampled(M):
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 3000 + M, a_dtype)
+    cols = synthetic.column_sample(N, 128, seed=M)
+    C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("sym,group,a_dtype", [(s, g, d) for s in (0, 1) for g in (32, 128) for d in (0, 1)])
+def test_gemm_format_variants_sampled(sym, group, a_dtype):
+    K = N = 8192
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("student_t", K, N, group, sym, 5)
+    for M in (1, 16, 256):
+        Ab, A = _acts(M, K, 4000 + M, a_dtype)
+        cols = synthetic.column_sample(N, 64, seed=M + group)
+        C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
+        torch.cuda.synchronize()
+        _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

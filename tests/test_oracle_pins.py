@@ -395,3 +395,37 @@ def test_quantized_layer_tracks_the_fp16_layer(oracle_mod):
     s = np.repeat(oracle_mod.decode16(scales), group, axis=0)
     bound = np.abs(a) @ (s / 2) * (1 + 2.0 ** -9)
     assert np.all(np.abs(Y - a @ W) <= bound)
+
+
+# ----------------------------------------------------------------------------- tiled layout
+def test_tiled_layout_positions_and_bijection(oracle_mod):
+    """The tiled buffer is a permutation of the plain words: each word lands once, at the
+    position the layout's definition gives (closed forms for chosen words)."""
+    K, N, group = 256, 384, 64
+    nwords = (K // 8) * N
+    codes = np.arange(nwords, dtype=np.int32).reshape(K // 8, N)   # word value = plain index
+    scales = np.arange((K // group) * N, dtype=np.uint16).reshape(K // group, N)
+    zeros = np.arange((K // group) * (N // 8), dtype=np.int32).reshape(K // group, N // 8)
+    buf = oracle_mod.repack(codes, scales, zeros, K, N, group, False)
+    off = oracle_mod.tiled_offsets(K, N, group, False)
+    words = buf[: off["codes_bytes"]].view(np.int32)
+    assert np.array_equal(np.sort(words), np.arange(nwords))        # a bijection
+    ktiles = K // 64
+    def plain(j, n):
+        return j * N + n
+    assert words[0] == plain(0, 0)
+    assert words[1] == plain(1, 0)          # four consecutive rows of one channel in 16 bytes
+    assert words[3] == plain(3, 0)
+    assert words[4] == plain(0, 1)          # then the next channel
+    assert words[512] == plain(4, 0)        # second half of the tile: rows 4..7
+    assert words[1024] == plain(8, 0)       # next tile along K
+    assert words[ktiles * 1024] == plain(0, 128)   # next 128 channels
+    assert words[ktiles * 1024 + 1024 + 512 + 4 * 5 + 2] == plain(8 + 4 + 2, 128 + 5)
+    assert off["scales"] % 256 == 0 and off["zeros"] % 256 == 0 and off["total"] % 256 == 0
+    assert off["scales"] >= off["codes_bytes"]
+    assert np.array_equal(buf[off["scales"]: off["scales"] + off["scales_bytes"]].view(np.uint16),
+                          scales.reshape(-1))
+    assert np.array_equal(buf[off["zeros"]: off["zeros"] + off["zeros_bytes"]].view(np.int32),
+                          zeros.reshape(-1))
+    offs = oracle_mod.tiled_offsets(K, N, group, True)
+    assert offs["zeros_bytes"] == 0

@@ -1,0 +1,177 @@
+// api.cu -- the C ABI of include/w4a16.h: host-side argument checks, the M-based dispatch and
+// the launches. Nothing here allocates device memory or synchronises the device.
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "tiled_layout.cuh"
+
+using namespace w4a16;
+
+namespace {
+
+bool valid_group(int group) { return group == 32 || group == 64 || group == 128; }
+
+int check_shape(int K, int N, int group) {
+    if (K <= 0 || N <= 0) return W4A16_EINVAL;
+    if (K % 8 != 0 || N % 8 != 0) return W4A16_EINVAL;
+    if (!valid_group(group)) return W4A16_EUNSUPPORTED;
+    if (K % group != 0) return W4A16_EINVAL;
+    return W4A16_OK;
+}
+
+// W4A16_FORCE_KERNEL=gemv|tc, read once.
+int forced_kernel() {
+    static int forced = -1;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        forced = W4A16_KERNEL_AUTO;
+        const char* e = getenv("W4A16_FORCE_KERNEL");
+        if (e && strcmp(e, "gemv") == 0) forced = W4A16_KERNEL_GEMV;
+        if (e && strcmp(e, "tc") == 0) forced = W4A16_KERNEL_TC;
+    });
+    return forced;
+}
+
+bool log_enabled() {
+    static bool on = false;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = getenv("W4A16_LOG");
+        on = e && e[0] == '1';
+    });
+    return on;
+}
+
+const char* kernel_name(int k) {
+    switch (k) {
+        case W4A16_KERNEL_GEMV: return "gemv";
+        case W4A16_KERNEL_TC: return "tc";
+        default: return "auto";
+    }
+}
+
+// The dispatch proper, without the environment override.
+int dispatch(int M, int N, int K, int group) {
+    (void)N;
+    (void)K;
+    (void)group;
+    (void)M;
+    return W4A16_KERNEL_GEMV;
+}
+
+}  // namespace
+
+extern "C" {
+
+W4A16_API int w4a16_version(void) { return 100; }
+
+W4A16_API const char* w4a16_status_str(int status) {
+    switch (status) {
+        case W4A16_OK: return "W4A16_OK";
+        case W4A16_EINVAL: return "W4A16_EINVAL";
+        case W4A16_EALIGN: return "W4A16_EALIGN";
+        case W4A16_EUNSUPPORTED: return "W4A16_EUNSUPPORTED";
+        case W4A16_ENONFINITE: return "W4A16_ENONFINITE";
+        case W4A16_EWORKSPACE: return "W4A16_EWORKSPACE";
+        case W4A16_ECUDA: return "W4A16_ECUDA";
+        case W4A16_ETIMEOUT: return "W4A16_ETIMEOUT";
+        default: return "W4A16_UNKNOWN";
+    }
+}
+
+W4A16_API int w4a16_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes,
+                             void* scales, int32_t* zeros, int* dev_status, void* stream) {
+    int st = check_shape(K, N, group);
+    if (st != W4A16_OK) return st;
+    if (sym != 0 && sym != 1) return W4A16_EINVAL;
+    if (!W || !codes || !scales) return W4A16_EINVAL;
+    if (sym ? zeros != nullptr : zeros == nullptr) return W4A16_EINVAL;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+        return W4A16_EALIGN;
+    return launch_quantize(W, K, N, group, sym, codes, scales, zeros, dev_status,
+                           static_cast<cudaStream_t>(stream));
+}
+
+W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym) {
+    if (check_shape(K, N, group) != W4A16_OK || (sym != 0 && sym != 1)) return 0;
+    if (N % kTileN != 0 || K % kTileK != 0) return 0;
+    return tiled_offsets(K, N, group, sym).total;
+}
+
+W4A16_API int w4a16_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K,
+                           int N, int group, int sym, void* tiled, void* stream) {
+    int st = check_shape(K, N, group);
+    if (st != W4A16_OK) return st;
+    if (sym != 0 && sym != 1) return W4A16_EINVAL;
+    if (N % kTileN != 0 || K % kTileK != 0) return W4A16_EUNSUPPORTED;
+    if (!codes || !scales || !tiled) return W4A16_EINVAL;
+    if (sym ? zeros != nullptr : zeros == nullptr) return W4A16_EINVAL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(tiled) || (zeros && !aligned16(zeros)))
+        return W4A16_EALIGN;
+    return launch_repack(codes, scales, zeros, K, N, group, sym, tiled,
+                         static_cast<cudaStream_t>(stream));
+}
+
+W4A16_API int w4a16_select_kernel(int M, int N, int K, int group) {
+    const int f = forced_kernel();
+    if (f != W4A16_KERNEL_AUTO) return f;
+    return dispatch(M, N, K, group);
+}
+
+W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group) {
+    if (M < 1 || check_shape(K, N, group) != W4A16_OK) return 0;
+    // the largest need over every kernel a call may run, so a forced kernel also fits
+    const GemvPlan p = plan_gemv_plain(M, N, K, group);
+    return p.ws_bytes;
+}
+
+W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* wq, int layout,
+                         const void* scales, const int32_t* zeros, int N, int group, int sym,
+                         void* C, void* workspace, size_t ws_bytes, int kernel, void* stream) {
+    int st = check_shape(K, N, group);
+    if (st != W4A16_OK) return st;
+    if (M < 1) return W4A16_EINVAL;
+    if (a_dtype != W4A16_F16 && a_dtype != W4A16_BF16) return W4A16_EINVAL;
+    if (layout != W4A16_LAYOUT_PLAIN && layout != W4A16_LAYOUT_TILED) return W4A16_EINVAL;
+    if (sym != 0 && sym != 1) return W4A16_EINVAL;
+    if (kernel != W4A16_KERNEL_AUTO && kernel != W4A16_KERNEL_GEMV && kernel != W4A16_KERNEL_TC)
+        return W4A16_EINVAL;
+    if (!A || !wq || !C) return W4A16_EINVAL;
+    if (layout == W4A16_LAYOUT_PLAIN) {
+        if (!scales) return W4A16_EINVAL;
+        if (sym ? zeros != nullptr : zeros == nullptr) return W4A16_EINVAL;
+        if (!aligned16(scales) || (zeros && !aligned16(zeros))) return W4A16_EALIGN;
+    } else if (N % kTileN != 0 || K % kTileK != 0) {
+        return W4A16_EUNSUPPORTED;
+    }
+    if (!aligned16(A) || !aligned16(wq) || !aligned16(C)) return W4A16_EALIGN;
+    const size_t need = w4a16_workspace_bytes(M, N, K, group);
+    if (ws_bytes < need || (need > 0 && !workspace)) return W4A16_EWORKSPACE;
+    if (workspace && !aligned16(workspace)) return W4A16_EALIGN;
+
+    const int chosen = kernel == W4A16_KERNEL_AUTO ? w4a16_select_kernel(M, N, K, group) : kernel;
+    if (log_enabled())
+        fprintf(stderr, "[w4a16] gemm M=%d N=%d K=%d g=%d sym=%d layout=%d -> %s\n", M, N, K, group,
+                sym, layout, kernel_name(chosen));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (chosen == W4A16_KERNEL_GEMV && layout == W4A16_LAYOUT_PLAIN) {
+        const GemvPlan p = plan_gemv_plain(M, N, K, group);
+        const size_t elt = 2;
+        for (int m0 = 0; m0 < M; m0 += p.mt) {
+            const int mc = (M - m0) < p.mt ? (M - m0) : p.mt;
+            st = launch_gemv_plain(static_cast<const char*>(A) + (size_t)m0 * K * elt, a_dtype, mc, K,
+                                   static_cast<const int32_t*>(wq), scales, zeros, N, group, sym,
+                                   static_cast<char*>(C) + (size_t)m0 * N * elt, workspace, p, s);
+            if (st != W4A16_OK) return st;
+        }
+        return W4A16_OK;
+    }
+    return W4A16_EUNSUPPORTED;
+}
+
+}  // extern "C"

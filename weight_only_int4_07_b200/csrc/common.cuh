@@ -1,0 +1,65 @@
+// common.cuh -- shared device/host helpers of the W4A16 CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "w4a16.h"
+
+namespace w4a16 {
+
+// 16-bit activation types and their conversions to/from FP32.
+template <typename T>
+struct Act;
+
+template <>
+struct Act<__half> {
+    static __device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+    static __device__ __forceinline__ __half from_f32(float x) { return __float2half_rn(x); }
+};
+
+template <>
+struct Act<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f32(float x) { return __float2bfloat16_rn(x); }
+};
+
+// First device-side error wins; the caller zeroes the status word.
+__device__ __forceinline__ void report_status(int* dev_status, int code) {
+    if (dev_status) atomicCAS(dev_status, 0, code);
+}
+
+// Nibble i of a packed word as an unsigned code 0..15.
+__device__ __forceinline__ int nibble_u(uint32_t w, int i) { return (int)((w >> (4 * i)) & 0xFu); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ECUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Kernel entry points implemented in the .cu files (host-side launchers).
+// ---------------------------------------------------------------------------------------------
+int launch_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes, void* scales,
+                    int32_t* zeros, int* dev_status, cudaStream_t stream);
+
+int launch_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
+                  int group, int sym, void* tiled, cudaStream_t stream);
+
+// Split-K GEMV plan: how the K dimension is cut and how much workspace that needs.
+struct GemvPlan {
+    int mt;              // rows of A per launch (template width), >= rows handled
+    int splits;          // K splits (grid.y)
+    int rows_per_split;  // packed rows (8 k each) per split
+    size_t ws_bytes;     // workspace for the partial sums of one launch
+};
+GemvPlan plan_gemv_plain(int M, int N, int K, int group);
+
+int launch_gemv_plain(const void* A, int a_dtype, int M, int K, const int32_t* codes,
+                      const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
+                      void* workspace, const GemvPlan& plan, cudaStream_t stream);
+
+}  // namespace w4a16

@@ -7,8 +7,8 @@ bit patterns of the 16-bit float type, so the two sides see identical bits.
 
 Distributions follow the workloads the layer is measured on:
   * weights ~ N(0, 0.02) in fp16;
-  * weights ~ N(0, 0.02) with a fixed fraction of entries (chosen by a seeded permutation)
-    multiplied by a constant (outliers);
+  * weights ~ N(0, 0.02) with a fixed fraction of entries (a seeded sample without
+    replacement) multiplied by a constant (outliers);
   * weights ~ 0.02 * Student-t(nu=5) in fp16;
   * activations ~ N(0, 1) in fp16 or bf16.
 """
@@ -39,7 +39,7 @@ def weights_outliers(K, N, seed, std=0.02, frac=0.001, mult=20.0):
     rng = _rng(seed)
     w = rng.standard_normal((K, N), dtype=np.float32) * np.float32(std)
     n_out = int(round(frac * K * N))
-    idx = rng.permutation(K * N)[:n_out]
+    idx = rng.choice(K * N, size=n_out, replace=False)
     w.reshape(-1)[idx] *= np.float32(mult)
     return _to_bits(w, F16)
 
