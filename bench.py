@@ -193,7 +193,7 @@ class DecodeStack:
         self.a_elems = sum(M * K for (_, K, _) in LLAMA8B_LINEARS) * layers
         self.c_elems = sum(M * N for (_, _, N) in LLAMA8B_LINEARS) * layers
         Ab = synthetic.activations(1, self.a_elems, seed + 100)
-        self.A_host = torch.from_numpy(Ab.view(np.int16)).view(torch.float16).pin_memory()
+        self.A_host = torch.from_numpy(Ab.view(np.int16).reshape(-1)).view(torch.float16).pin_memory()
         self.A = self.A_host.to(dev)
         self.C = torch.empty(self.c_elems, dtype=torch.float16, device=dev)
         self.C_host = torch.empty(self.c_elems, dtype=torch.float16).pin_memory()
@@ -225,12 +225,12 @@ class DecodeStack:
             self.gemm(w, A, C)
 
 
-def tiled_supported(torch, native, qw):
-    """Whether the library runs the tiled layout (probed with one small call)."""
+def tiled_supported(torch, native, qw, M=1):
+    """Whether the library runs the tiled layout for M rows (probed with one call)."""
     K, N, codes, scales, zeros = qw
     try:
         t = native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM)
-        A = torch.zeros((1, K), dtype=torch.float16, device=codes.device)
+        A = torch.zeros((M, K), dtype=torch.float16, device=codes.device)
         native.w4a16_gemm(A, t, None, None, N, GROUP, SYM, layout=native.LAYOUT_TILED)
         torch.cuda.synchronize()
         return True
@@ -241,20 +241,36 @@ def tiled_supported(torch, native, qw):
 
 
 def count_graph_kernels(graph):
-    """Kernel nodes in a captured torch CUDA graph (None when the graph cannot be inspected)."""
+    """Kernel nodes in a captured CUDA graph, through the driver API (None when unavailable)."""
     try:
-        from cuda.bindings import runtime as cudart
+        import ctypes
+
+        cu = ctypes.CDLL("libcuda.so.1")
         raw = graph.raw_cuda_graph()
-        err, nodes, n = cudart.cudaGraphGetNodes(raw, 0)
-        err, nodes, n = cudart.cudaGraphGetNodes(raw, n)
+        handle = ctypes.c_void_p(int(raw))
+        n = ctypes.c_size_t(0)
+        if cu.cuGraphGetNodes(handle, None, ctypes.byref(n)) != 0:
+            return None
+        nodes = (ctypes.c_void_p * n.value)()
+        if cu.cuGraphGetNodes(handle, nodes, ctypes.byref(n)) != 0:
+            return None
         count = 0
-        for node in nodes:
-            err, typ = cudart.cudaGraphNodeGetType(node)
-            if typ == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel:
-                count += 1
+        for i in range(n.value):
+            t = ctypes.c_int(-1)
+            if cu.cuGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) != 0:
+                return None
+            count += int(t.value == 0)  # CU_GRAPH_NODE_TYPE_KERNEL
         return count
     except Exception:
         return None
+
+
+def new_graph(torch):
+    """A torch CUDA graph that keeps its cudaGraph_t after instantiation (for node counting)."""
+    try:
+        return torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        return torch.cuda.CUDAGraph()
 
 
 def time_graph(torch, graph, steps, world, dev):
@@ -326,7 +342,7 @@ def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
     W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).to(dev)
     codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
     del W
-    use_tiled = tiled_supported(torch, native, (K, N, codes, scales, zeros))
+    use_tiled = tiled_supported(torch, native, (K, N, codes, scales, zeros), M)
     ws_need = native.w4a16_workspace_bytes(M, N, K, GROUP)
     ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
     if use_tiled:
@@ -364,7 +380,7 @@ def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
     torch.cuda.synchronize()
     durs = [s.elapsed_time(e) for (s, e) in evs]
     ms = statistics.mean(durs)
-    kernel = native.w4a16_select_kernel(M, N, K, GROUP)
+    kernel = native.w4a16_select_kernel(M, N, K, GROUP) if use_tiled else native.KERNEL_GEMV
     return {"M": M, "K": K, "N": N, "ms": ms, "tflops": gemm_flops(M, K, N) / (ms * 1e-3) / 1e12,
             "kernel": {1: "gemv", 2: "tc"}.get(kernel, str(kernel)), "dtype": "bf16",
             "bytes": algorithmic_bytes(M, K, N), "launches": len(durs),
@@ -379,9 +395,8 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def oracle_sample(synthetic, seed, threads, budget_s=15.0, min_reps=1):
-    """The FP64 oracle's layer throughput on one Llama-3-8B layer (all four linears, all
-    columns, M = 1, fp16), repeated while under budget. Returns (GB/s, seconds, reps)."""
+def oracle_prepare(synthetic, seed, threads):
+    """One Llama-3-8B-shaped layer quantized by the oracle, with one activation row per linear."""
     import oracle
 
     packed = []
@@ -390,16 +405,33 @@ def oracle_sample(synthetic, seed, threads, budget_s=15.0, min_reps=1):
         st, c, s, z = oracle.quantize(Wb, GROUP, SYM, nthreads=threads)
         Ab = synthetic.activations(1, K, seed + 200 + i)
         packed.append((K, N, c, s, z, Ab))
+    return packed
+
+
+def oracle_pass(packed, threads):
+    """One pass of the FP64 oracle over the layer's four linears (all columns, M = 1).
+    Returns (algorithmic bytes, seconds)."""
+    import oracle
+
+    nbytes, secs = 0, 0.0
+    for (K, N, c, s, z, Ab) in packed:
+        t0 = time.perf_counter()
+        oracle.linear(Ab, 0, c, s, z, N, GROUP, SYM, nthreads=threads)
+        secs += time.perf_counter() - t0
+        nbytes += algorithmic_bytes(1, K, N)
+    return nbytes, secs
+
+
+def oracle_sample(synthetic, seed, threads, budget_s=15.0):
+    """The oracle's throughput, passes repeated while under the time budget.
+    Returns (GB/s, seconds, passes)."""
+    packed = oracle_prepare(synthetic, seed, threads)
     reps, total, nbytes = 0, 0.0, 0
-    while reps < min_reps or total < budget_s:
-        for (K, N, c, s, z, Ab) in packed:
-            t0 = time.perf_counter()
-            oracle.linear(Ab, 0, c, s, z, N, GROUP, SYM, nthreads=threads)
-            total += time.perf_counter() - t0
-            nbytes += algorithmic_bytes(1, K, N)
+    while reps < 1 or total < budget_s:
+        b, t = oracle_pass(packed, threads)
+        nbytes += b
+        total += t
         reps += 1
-        if total > budget_s:
-            break
     return nbytes / total / 1e9, total, reps
 
 
@@ -411,14 +443,16 @@ def run_reference(args):
     from weight_only_int4_07_b200 import synthetic
 
     threads = host_cores()
-    per_step = []
+    packed = oracle_prepare(synthetic, 11, threads)
     for _ in range(args.warmup):
-        oracle_sample(synthetic, 11, threads, budget_s=0.0)
+        oracle_pass(packed, threads)
+    tot_b, tot_s = 0, 0.0
     for _ in range(args.steps):
-        gbs, secs, reps = oracle_sample(synthetic, 11, threads, budget_s=0.0)
-        per_step.append((gbs, secs))
-    value = statistics.mean(g for g, _ in per_step)
-    ms = 1e3 * statistics.mean(s for _, s in per_step)
+        b, t = oracle_pass(packed, threads)
+        tot_b += b
+        tot_s += t
+    value = tot_b / tot_s / 1e9
+    ms = 1e3 * tot_s / args.steps
     sample = ("one Llama-3-8B-shaped layer per step: the four decode linears (4096x6144, 4096x4096, "
               "4096x28672, 14336x4096), all columns, M=1, g128 asym, fp16; FP64 oracle")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
@@ -465,11 +499,16 @@ def run_ours(args):
     for _ in range(max(args.warmup, 1)):
         stack.step()
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
+    graph = new_graph(torch)
     with torch.cuda.graph(graph):
         stack.step()
     torch.cuda.synchronize()
     kernels_per_step = count_graph_kernels(graph)
+    if hasattr(graph, "instantiate"):
+        try:
+            graph.instantiate()
+        except RuntimeError:
+            pass
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()

@@ -125,7 +125,10 @@ W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);
  * (4 KiB) holding word (j, n) of the plain layout at offset
  *     ((j % 8) / 4) * 512 + (n % 128) * 4 + (j % 4)            (j = 8 c + j % 8)
  * so that one 16-byte vector holds four consecutive words along K of one output channel, and a
- * warp's 32 consecutive output channels read 512 contiguous bytes. Scales and zeros follow the
+ * warp's 32 consecutive output channels read 512 contiguous bytes. Each word is re-encoded:
+ * nibble slot p (bits 4p..4p+3, p = 0..3) holds the code of element 2p (k = 8j + 2p) and slot
+ * p + 4 that of element 2p + 1; symmetric codes are stored offset-binary, q + 8, so that both
+ * schemes dequantize as (u - z) * s with z = 8 for the symmetric one. Scales and zeros follow the
  * codes in the same buffer, in the plain layouts [K/g, N] fp16 and [K/g, N/8] int32 (asym),
  * each starting on a 256-byte boundary.
  * Requires N % 128 == 0 and K % 64 == 0 (else W4A16_EUNSUPPORTED).
@@ -168,14 +171,17 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
  *   workspace  device scratch of at least w4a16_workspace_bytes(M, N, K, group) bytes (NULL if 0).
  *              Calls that share one workspace must be ordered on the GPU (same stream).
  *   ws_bytes   size of workspace.
- *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC.
+ *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC. The tensor-core
+ *              kernel reads the TILED layout only (PLAIN with W4A16_KERNEL_TC is unsupported).
+ *   dev_status device int or NULL: set to W4A16_ETIMEOUT if a bounded on-device wait gave up
+ *              (the output is then unspecified; the device stays usable).
  *   stream     cudaStream_t.
  * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
  * W4A16_ECUDA.
  */
 W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* wq, int layout,
                const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
-               void* workspace, size_t ws_bytes, int kernel, void* stream);
+               void* workspace, size_t ws_bytes, int kernel, int* dev_status, void* stream);
 
 /* w4a16_status_str -- a static, human-readable name for a status code. */
 W4A16_API const char* w4a16_status_str(int status);

@@ -329,7 +329,10 @@ int w4o_max_threads(void) {
  * tiles of 128 output channels x 64 input channels (8 packed rows); tile (t, c) has index
  * t * (K/64) + c and holds 1024 words; plain word (j, n) sits at
  *   ((j mod 8) div 4) * 512 + (n mod 128) * 4 + (j mod 4)
- * inside its tile. Scales (plain [K/g, N] fp16) and zeros (plain [K/g, N/8] int32, asym only)
+ * inside its tile, with its codes re-ordered: nibble slot p (p = 0..3) holds the code of element
+ * 2p and slot p + 4 that of element 2p + 1 (element e = row k - 8j of the word); symmetric codes
+ * are stored offset-binary, q + 8 (zero-point 8).
+ * Scales (plain [K/g, N] fp16) and zeros (plain [K/g, N/8] int32, asym only)
  * follow, each region starting at a multiple of 256 bytes. Padding bytes are left zero.
  * (The pages ask for a pre-permuted layout -- "INT4 and Low-Bit Inference", section 5
  * "The kernel is half the story" -- but leave its form open; this one is the library's.)
@@ -365,7 +368,15 @@ int w4o_repack(const int32_t* codes, const uint16_t* scales, const int32_t* zero
                 for (long nl = 0; nl < 128; ++nl) {
                     const long j = 8 * c + jl, n = 128 * t + nl;
                     const long pos = (t * ktiles + c) * 1024 + (jl / 4) * 512 + nl * 4 + (jl % 4);
-                    tiled[pos] = codes[j * N + n];
+                    const uint32_t w = (uint32_t)codes[j * N + n];
+                    uint32_t t = 0;
+                    for (int e = 0; e < 8; ++e) {
+                        uint32_t u = (w >> (4 * e)) & 0xFu;            /* element e */
+                        if (sym) u = (u + 8u) & 0xFu;                  /* q + 8 for q in -8..7 */
+                        const int slot = (e % 2 == 0) ? e / 2 : 4 + e / 2;
+                        t |= u << (4 * slot);
+                    }
+                    tiled[pos] = (int32_t)t;
                 }
     memcpy(out + off[2], scales, (size_t)off[3]);
     if (!sym) memcpy(out + off[4], zeros, (size_t)off[5]);

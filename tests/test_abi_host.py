@@ -97,7 +97,8 @@ MIS = ctypes.c_void_p((5 << 20) + 8)
 
 def _gemm(L, A=A16, dt=0, M=1, K=256, wq=B16, layout=0, scales=C16, zeros=D16, N=256, g=128,
           sym=0, C=A16, ws=None, wsb=1 << 30, kernel=0):
-    return L.w4a16_gemm(A, dt, M, K, wq, layout, scales, zeros, N, g, sym, C, ws, wsb, kernel, None)
+    return L.w4a16_gemm(A, dt, M, K, wq, layout, scales, zeros, N, g, sym, C, ws, wsb, kernel, None,
+                        None)
 
 
 def test_gemm_rejects_bad_arguments(L):

@@ -252,3 +252,92 @@ def test_gemm_format_variants_sampled(sym, group, a_dtype):
         C = native.w4a16_gemm(A, gc, gs, gz, N, group, sym)
         torch.cuda.synchronize()
         _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+# ----------------------------------------------------------------------------- tiled layout + tcgen05
+def _tiled(kind, K, N, group, sym, seed):
+    key = ("T", kind, K, N, group, sym, seed)
+    if key not in _cache:
+        Wb, o, (gc, gs, gz) = _quantized(kind, K, N, group, sym, seed)
+        _cache[key] = (Wb, o, native.w4a16_repack(gc, gs, gz, K, N, group, sym))
+    return _cache[key]
+
+
+TILED_GEMM = [
+    # M, K, N, group, sym, a_dtype
+    (1, 512, 256, 128, 0, 0),
+    (16, 512, 256, 32, 1, 1),
+    (17, 1024, 384, 64, 0, 0),
+    (32, 768, 128, 32, 0, 1),
+    (33, 1024, 256, 128, 1, 0),
+    (64, 2048, 512, 128, 0, 1),
+    (100, 512, 384, 64, 1, 1),
+    (128, 1024, 256, 32, 0, 0),
+    (200, 512, 128, 128, 0, 1),
+    (256, 1024, 384, 64, 0, 0),
+    (300, 512, 256, 32, 1, 1),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", TILED_GEMM)
+@pytest.mark.parametrize("kernel", [native.KERNEL_TC, native.KERNEL_AUTO])
+def test_gemm_tiled_full_output(M, K, N, group, sym, a_dtype, kernel):
+    kind = "student_t" if sym else "normal"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 60 + K + N)
+    Ab, A = _acts(M, K, 500 + M, a_dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                              kernel=kernel, dev_status=status)
+    except native.W4A16Error as e:
+        # the AUTO dispatch may pick a kernel that has no tiled variant for this M
+        assert kernel == native.KERNEL_AUTO and e.status == native.EUNSUPPORTED
+        return
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+@pytest.mark.parametrize("sym", [0, 1])
+def test_gemm_tc_unit_rows_return_dequantized_rows(a_dtype, sym):
+    K, N, group = 512, 256, 64
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
+    rows = [0, 1, 7, 8, 63, 64, 200, 511] * 5   # 40 rows -> the tensor-core path
+    Ab = np.zeros((len(rows), K), dtype=np.uint16)
+    one = 0x3C00 if a_dtype == 0 else 0x3F80
+    for i, k in enumerate(rows):
+        Ab[i, k] = one
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_TC)
+    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
+    expect = oracle.decode16(oracle.encode16(What[rows], a_dtype), a_dtype)   # one rounding
+    got = oracle.decode16(_to_np16(C), a_dtype)
+    assert np.array_equal(got, expect)
+
+
+@pytest.mark.parametrize("M", [32, 64, 256, 512])
+def test_gemm_tc_sweep_shape_sampled(M):
+    """The (8192, 28672) sweep layer in the launch configuration the benchmark times."""
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 6000 + M, a_dtype)
+    cols = synthetic.column_sample(N, 96, seed=M + 1)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("sym,group,a_dtype", [(s, g, d) for s in (0, 1) for g in (32, 128) for d in (0, 1)])
+def test_gemm_tc_format_variants_sampled(sym, group, a_dtype):
+    K = N = 8192
+    Wb, (oc, os_, oz), tiled = _tiled("student_t", K, N, group, sym, 5)
+    for M in (16, 256):
+        Ab, A = _acts(M, K, 7000 + M, a_dtype)
+        cols = synthetic.column_sample(N, 64, seed=M + group + 1)
+        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                              kernel=native.KERNEL_TC)
+        torch.cuda.synchronize()
+        _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

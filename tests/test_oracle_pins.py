@@ -398,29 +398,52 @@ def test_quantized_layer_tracks_the_fp16_layer(oracle_mod):
 
 
 # ----------------------------------------------------------------------------- tiled layout
+def _slots(word):
+    """The eight nibbles of a word, slot 0 first."""
+    return [(int(word) >> (4 * i)) & 0xF for i in range(8)]
+
+
 def test_tiled_layout_positions_and_bijection(oracle_mod):
     """The tiled buffer is a permutation of the plain words: each word lands once, at the
-    position the layout's definition gives (closed forms for chosen words)."""
+    position the layout's definition gives (closed forms for chosen words), with its codes in
+    slot order (e0, e2, e4, e6, e1, e3, e5, e7)."""
     K, N, group = 256, 384, 64
-    nwords = (K // 8) * N
-    codes = np.arange(nwords, dtype=np.int32).reshape(K // 8, N)   # word value = plain index
+    rows = K // 8
+    nwords = rows * N
+    # every plain word carries its own index in bits 8..31 and the element number in the
+    # low byte pattern 0x10 (element 0 = 0, element 1 = 1): make element e's nibble = e
+    rng = np.random.default_rng(17)
+    codes = rng.integers(-2**31, 2**31, size=(rows, N), dtype=np.int64).astype(np.int32)
     scales = np.arange((K // group) * N, dtype=np.uint16).reshape(K // group, N)
     zeros = np.arange((K // group) * (N // 8), dtype=np.int32).reshape(K // group, N // 8)
     buf = oracle_mod.repack(codes, scales, zeros, K, N, group, False)
     off = oracle_mod.tiled_offsets(K, N, group, False)
     words = buf[: off["codes_bytes"]].view(np.int32)
-    assert np.array_equal(np.sort(words), np.arange(nwords))        # a bijection
+    assert words.size == nwords
     ktiles = K // 64
-    def plain(j, n):
-        return j * N + n
-    assert words[0] == plain(0, 0)
-    assert words[1] == plain(1, 0)          # four consecutive rows of one channel in 16 bytes
-    assert words[3] == plain(3, 0)
-    assert words[4] == plain(0, 1)          # then the next channel
-    assert words[512] == plain(4, 0)        # second half of the tile: rows 4..7
-    assert words[1024] == plain(8, 0)       # next tile along K
-    assert words[ktiles * 1024] == plain(0, 128)   # next 128 channels
-    assert words[ktiles * 1024 + 1024 + 512 + 4 * 5 + 2] == plain(8 + 4 + 2, 128 + 5)
+
+    def plain_elems(j, n):
+        return _slots(np.uint32(codes[j, n]))
+
+    def check(pos, j, n):
+        e = plain_elems(j, n)
+        assert _slots(np.uint32(words[pos])) == [e[0], e[2], e[4], e[6], e[1], e[3], e[5], e[7]]
+
+    check(0, 0, 0)
+    check(1, 1, 0)           # four consecutive rows of one channel in 16 bytes
+    check(3, 3, 0)
+    check(4, 0, 1)           # then the next channel
+    check(512, 4, 0)         # second half of the tile: rows 4..7
+    check(1024, 8, 0)        # next tile along K
+    check(ktiles * 1024, 0, 128)   # next 128 channels
+    check(ktiles * 1024 + 1024 + 512 + 4 * 5 + 2, 8 + 4 + 2, 128 + 5)
+    # a bijection: decode every tiled word back and compare the multiset of plain words
+    def decode(t):
+        s_ = _slots(np.uint32(t))
+        e = [s_[0], s_[4], s_[1], s_[5], s_[2], s_[6], s_[3], s_[7]]
+        return sum(v << (4 * i) for i, v in enumerate(e))
+    back = np.array(sorted(decode(t) for t in words), dtype=np.int64)
+    assert np.array_equal(back, np.sort((codes.astype(np.int64) & 0xFFFFFFFF).reshape(-1)))
     assert off["scales"] % 256 == 0 and off["zeros"] % 256 == 0 and off["total"] % 256 == 0
     assert off["scales"] >= off["codes_bytes"]
     assert np.array_equal(buf[off["scales"]: off["scales"] + off["scales_bytes"]].view(np.uint16),
@@ -429,3 +452,19 @@ def test_tiled_layout_positions_and_bijection(oracle_mod):
                           zeros.reshape(-1))
     offs = oracle_mod.tiled_offsets(K, N, group, True)
     assert offs["zeros_bytes"] == 0
+
+
+def test_tiled_layout_symmetric_is_offset_binary(oracle_mod):
+    """Symmetric codes -8..7 are stored as q + 8 (0..15) in the tiled buffer."""
+    K, N, group = 64, 128, 32
+    q = np.tile(np.arange(-8, 8), 4 * N // 16 * K // 4)[: K * N].reshape(K, N)
+    words = np.zeros((K // 8, N), dtype=np.int64)
+    for k in range(K):
+        words[k // 8] |= (q[k] & 0xF).astype(np.int64) << (4 * (k % 8))
+    codes = words.astype(np.uint32).view(np.int32)
+    scales = np.full((K // group, N), 0x3C00, dtype=np.uint16)
+    buf = oracle_mod.repack(codes, scales, None, K, N, group, True)
+    t = buf[: K * N // 2].view(np.int32)
+    # word (j = 0, n = 0) sits at position 0: its slots hold q[0, 0..7 even], q[.. odd] + 8
+    e = [q[k, 0] + 8 for k in range(8)]
+    assert _slots(np.uint32(t[0])) == [e[0], e[2], e[4], e[6], e[1], e[3], e[5], e[7]]

@@ -54,13 +54,14 @@ const char* kernel_name(int k) {
     }
 }
 
-// The dispatch proper, without the environment override.
+// The dispatch proper, without the environment override. At small M the layer is bound by the
+// weight stream and the split-K CUDA-core GEMV serves it; from M = 32 the tensor-core GEMM takes
+// over (it needs the tiled layout).
 int dispatch(int M, int N, int K, int group) {
     (void)N;
     (void)K;
     (void)group;
-    (void)M;
-    return W4A16_KERNEL_GEMV;
+    return M >= 32 ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
 }
 
 }  // namespace
@@ -131,7 +132,8 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group) {
 
 W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* wq, int layout,
                          const void* scales, const int32_t* zeros, int N, int group, int sym,
-                         void* C, void* workspace, size_t ws_bytes, int kernel, void* stream) {
+                         void* C, void* workspace, size_t ws_bytes, int kernel, int* dev_status,
+                         void* stream) {
     int st = check_shape(K, N, group);
     if (st != W4A16_OK) return st;
     if (M < 1) return W4A16_EINVAL;
@@ -153,7 +155,9 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
     if (ws_bytes < need || (need > 0 && !workspace)) return W4A16_EWORKSPACE;
     if (workspace && !aligned16(workspace)) return W4A16_EALIGN;
 
-    const int chosen = kernel == W4A16_KERNEL_AUTO ? w4a16_select_kernel(M, N, K, group) : kernel;
+    int chosen = kernel == W4A16_KERNEL_AUTO ? w4a16_select_kernel(M, N, K, group) : kernel;
+    // the plain layout has only the CUDA-core kernel
+    if (kernel == W4A16_KERNEL_AUTO && layout == W4A16_LAYOUT_PLAIN) chosen = W4A16_KERNEL_GEMV;
     if (log_enabled())
         fprintf(stderr, "[w4a16] gemm M=%d N=%d K=%d g=%d sym=%d layout=%d -> %s\n", M, N, K, group,
                 sym, layout, kernel_name(chosen));
@@ -170,6 +174,9 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
             if (st != W4A16_OK) return st;
         }
         return W4A16_OK;
+    }
+    if (chosen == W4A16_KERNEL_TC && layout == W4A16_LAYOUT_TILED) {
+        return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
     }
     return W4A16_EUNSUPPORTED;
 }

@@ -62,4 +62,7 @@ int launch_gemv_plain(const void* A, int a_dtype, int M, int K, const int32_t* c
                       const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
                       void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
+int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                   void* C, int* dev_status, cudaStream_t stream);
+
 }  // namespace w4a16

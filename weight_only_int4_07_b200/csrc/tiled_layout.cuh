@@ -17,6 +17,20 @@ __host__ __device__ __forceinline__ size_t tiled_word_offset(int j, int n, int K
     return tile * kTileWords + (size_t)((jl / 4) * 512 + nl * 4 + (jl % 4));
 }
 
+// Re-encoding of one plain word (nibble i = element i) for the tiled layout: slot p <- element
+// 2p, slot p + 4 <- element 2p + 1; symmetric codes become offset-binary (two's complement
+// nibble XOR 8 = q + 8).
+__host__ __device__ __forceinline__ uint32_t tiled_encode_word(uint32_t w, int sym) {
+    if (sym) w ^= 0x88888888u;
+    uint32_t t = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        t |= ((w >> (8 * p)) & 0xFu) << (4 * p);             // element 2p
+        t |= ((w >> (8 * p + 4)) & 0xFu) << (16 + 4 * p);    // element 2p + 1
+    }
+    return t;
+}
+
 struct TiledOffsets {
     size_t codes, codes_bytes;
     size_t scales, scales_bytes;

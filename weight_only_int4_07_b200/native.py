@@ -62,7 +62,7 @@ def lib():
     L.w4a16_workspace_bytes.restype = S
     L.w4a16_select_kernel.argtypes = [I, I, I, I]
     L.w4a16_select_kernel.restype = I
-    L.w4a16_gemm.argtypes = [P, I, I, I, P, I, P, P, I, I, I, P, P, S, I, P]
+    L.w4a16_gemm.argtypes = [P, I, I, I, P, I, P, P, I, I, I, P, P, S, I, P, P]
     L.w4a16_gemm.restype = I
     L.w4a16_status_str.argtypes = [I]
     L.w4a16_status_str.restype = ctypes.c_char_p
@@ -138,7 +138,7 @@ def w4a16_select_kernel(M, N, K, group) -> int:
 
 
 def w4a16_gemm(A, wq, scales, zeros, N, group, sym, layout=LAYOUT_PLAIN, C=None, workspace=None,
-               kernel=KERNEL_AUTO):
+               kernel=KERNEL_AUTO, dev_status=None):
     """C[M, N] = A[M, K] . dequant(W) with FP32 accumulation; C in the dtype of A."""
     M, K = A.shape
     a_dtype = _DTYPES[A.dtype]
@@ -150,6 +150,6 @@ def w4a16_gemm(A, wq, scales, zeros, N, group, sym, layout=LAYOUT_PLAIN, C=None,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().w4a16_gemm(_ptr(A), a_dtype, M, K, _ptr(wq), int(layout), _ptr(scales), _ptr(zeros),
                           N, group, int(sym), _ptr(C), _ptr(workspace), ws_bytes, int(kernel),
-                          _stream())
+                          _ptr(dev_status), _stream())
     _check("w4a16_gemm", st)
     return C
