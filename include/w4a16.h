@@ -183,6 +183,34 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
                const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
                void* workspace, size_t ws_bytes, int kernel, int* dev_status, void* stream);
 
+/*
+ * w4a16_gemm_noalloc -- w4a16_gemm for callers that cannot allocate device memory.
+ *   (The pages have no counterpart: this is a convenience of this library.)
+ *   w4a16_gemm needs a caller-provided workspace for its split-K partial sums. Callers that have
+ *   no way to provide one -- for example a plugin inside a host application that owns every
+ *   device allocation, or a latency-critical loop that must never call cudaMalloc because it can
+ *   block and synchronise the device -- call this instead. It runs the plain-layout split-K
+ *   CUDA-core GEMV with its partial sums in one static 8 MiB device array of this library,
+ *   reserved on every GPU that loads the library until the process exits; it calls no
+ *   cudaMalloc, cudaFree or other allocating routine.
+ * Limits and sharing
+ *   - The call's partial sums, splits x min(M, 16) x N FP32 values (see w4a16_workspace_bytes),
+ *     must fit in 8 MiB; a larger call returns W4A16_EWORKSPACE and launches nothing.
+ *   - Every call on a device uses the same array, which keeps the last call's contents (nothing
+ *     in it needs to start at zero). Calls that can overlap on the GPU -- on different streams,
+ *     or from different host threads -- race on it: order them on one stream.
+ *   - The first call on each device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call before any stream
+ *     capture begins.
+ * Arguments as w4a16_gemm with layout W4A16_LAYOUT_PLAIN (codes [K/8, N], scales [K/g, N],
+ * zeros [K/g, N/8] or NULL when sym), without workspace, kernel choice or dev_status.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
+ * W4A16_ECUDA.
+ */
+W4A16_API int w4a16_gemm_noalloc(const void* A, int a_dtype, int M, int K, const int32_t* codes,
+                                 const void* scales, const int32_t* zeros, int N, int group, int sym,
+                                 void* C, void* stream);
+
 /* w4a16_status_str -- a static, human-readable name for a status code. */
 W4A16_API const char* w4a16_status_str(int status);
 

@@ -153,3 +153,26 @@ def w4a16_gemm(A, wq, scales, zeros, N, group, sym, layout=LAYOUT_PLAIN, C=None,
                           _ptr(dev_status), _stream())
     _check("w4a16_gemm", st)
     return C
+
+
+_noalloc_ready = False
+
+
+def w4a16_gemm_noalloc(A, codes, scales, zeros, N, group, sym, C=None):
+    """C[M, N] = A[M, K] . dequant(W) for callers that cannot allocate device memory: the split-K
+    partial sums live in the library's static scratch (see include/w4a16.h for its limit and
+    for why calls that overlap on the GPU race)."""
+    global _noalloc_ready
+    L = lib()
+    if not _noalloc_ready:
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.w4a16_gemm_noalloc.argtypes = [P, I, I, I, P, P, P, I, I, I, P, P]
+        L.w4a16_gemm_noalloc.restype = I
+        _noalloc_ready = True
+    M, K = A.shape
+    if C is None:
+        C = torch.empty((M, N), dtype=A.dtype, device=A.device)
+    st = L.w4a16_gemm_noalloc(_ptr(A), _DTYPES[A.dtype], M, K, _ptr(codes), _ptr(scales), _ptr(zeros),
+                              N, group, int(sym), _ptr(C), _stream())
+    _check("w4a16_gemm_noalloc", st)
+    return C
