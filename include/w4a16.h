@@ -77,8 +77,10 @@ typedef enum {
 /* Kernel family chosen by the M-based dispatch (see w4a16_select_kernel). */
 typedef enum {
     W4A16_KERNEL_AUTO = 0,    /* let the dispatch decide                                      */
-    W4A16_KERNEL_GEMV = 1,    /* split-K CUDA-core GEMV / skinny GEMM, M <= 16                */
-    W4A16_KERNEL_TC = 2       /* tcgen05 tensor-core GEMM with TMEM accumulators              */
+    W4A16_KERNEL_GEMV = 1,    /* split-K CUDA-core GEMV (plain layout), any M                 */
+    W4A16_KERNEL_TC = 2,      /* tcgen05 tensor-core GEMM, TMEM accumulator (tiled layout)     */
+    W4A16_KERNEL_SKINNY = 3   /* split-K tcgen05 kernel for M <= 16, exact integer weights in
+                                 TMEM, per-group FP32 scaling, cluster reduction (tiled layout) */
 } w4a16_kernel;
 
 /*
@@ -146,10 +148,11 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
 
 /*
  * w4a16_select_kernel -- the M-based dispatch, as a pure host function: returns the
- * w4a16_kernel that w4a16_gemm(..., W4A16_KERNEL_AUTO) runs for this shape. Small M is bound
- * by the weight stream and goes to the split-K GEMV; larger M goes to the tensor-core GEMM
- * ("INT8 vs INT4 Quantization, in depth", section "Two regimes: waiting for memory, waiting
- * for math"). The environment variable W4A16_FORCE_KERNEL=gemv|tc overrides the choice.
+ * w4a16_kernel that w4a16_gemm(..., W4A16_KERNEL_AUTO) runs on the tiled layout for this shape.
+ * Small M is bound by the weight stream and goes to the split-K skinny kernel; larger M goes to
+ * the tensor-core GEMM ("INT8 vs INT4 Quantization, in depth", section "Two regimes: waiting for
+ * memory, waiting for math"). The plain layout always runs the CUDA-core GEMV.
+ * The environment variable W4A16_FORCE_KERNEL=gemv|tc|skinny overrides the choice.
  */
 W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
 
@@ -171,8 +174,9 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
  *   workspace  device scratch of at least w4a16_workspace_bytes(M, N, K, group) bytes (NULL if 0).
  *              Calls that share one workspace must be ordered on the GPU (same stream).
  *   ws_bytes   size of workspace.
- *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC. The tensor-core
- *              kernel reads the TILED layout only (PLAIN with W4A16_KERNEL_TC is unsupported).
+ *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC /
+ *              W4A16_KERNEL_SKINNY. GEMV reads the PLAIN layout only; TC and SKINNY read the TILED
+ *              layout only; SKINNY needs M <= 16. Other combinations return W4A16_EUNSUPPORTED.
  *   dev_status device int or NULL: set to W4A16_ETIMEOUT if a bounded on-device wait gave up
  *              (the output is then unspecified; the device stays usable).
  *   stream     cudaStream_t.

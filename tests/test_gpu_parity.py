@@ -334,10 +334,147 @@ def test_gemm_tc_sweep_shape_sampled(M):
 def test_gemm_tc_format_variants_sampled(sym, group, a_dtype):
     K = N = 8192
     Wb, (oc, os_, oz), tiled = _tiled("student_t", K, N, group, sym, 5)
-    for M in (16, 256):
+    for M, kernel in ((16, native.KERNEL_TC), (256, native.KERNEL_TC), (1, native.KERNEL_SKINNY),
+                      (16, native.KERNEL_SKINNY)):
         Ab, A = _acts(M, K, 7000 + M, a_dtype)
         cols = synthetic.column_sample(N, 64, seed=M + group + 1)
         C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                              kernel=native.KERNEL_TC)
+                              kernel=kernel)
         torch.cuda.synchronize()
         _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+# ----------------------------------------------------------------------------- tiled layout + skinny tcgen05
+SKINNY_GEMM = [
+    # M, K, N, group, sym, a_dtype    (splits follow from N, K and the group)
+    (1, 128, 128, 128, 0, 0),         # one unit: no split
+    (1, 512, 256, 128, 0, 0),         # the tiny configuration
+    (2, 512, 256, 32, 1, 1),
+    (3, 1024, 384, 64, 0, 0),
+    (5, 768, 128, 32, 0, 1),
+    (8, 2048, 512, 128, 1, 0),
+    (13, 1024, 256, 64, 1, 1),
+    (16, 4096, 1024, 128, 0, 1),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SKINNY_GEMM)
+def test_gemm_skinny_full_output(M, K, N, group, sym, a_dtype):
+    kind = "student_t" if sym else "normal"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 70 + K + N)
+    Ab, A = _acts(M, K, 800 + M, a_dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_SKINNY, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+@pytest.mark.parametrize("sym", [0, 1])
+def test_gemm_skinny_unit_rows_return_dequantized_rows(a_dtype, sym):
+    K, N, group = 512, 256, 64
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
+    rows = [0, 7, 8, 63, 64, 200, 300, 511, 1, 2, 3, 130, 257, 384, 450, 509]   # 16 rows
+    Ab = np.zeros((len(rows), K), dtype=np.uint16)
+    one = 0x3C00 if a_dtype == 0 else 0x3F80
+    for i, k in enumerate(rows):
+        Ab[i, k] = one
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_SKINNY)
+    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
+    expect = oracle.decode16(oracle.encode16(What[rows], a_dtype), a_dtype)   # one rounding
+    got = oracle.decode16(_to_np16(C), a_dtype)
+    assert np.array_equal(got, expect)
+
+
+def test_gemm_skinny_zero_weights_give_zero():
+    K, N, group = 1024, 256, 32
+    W = torch.zeros((K, N), dtype=torch.float16, device="cuda")
+    for sym in (0, 1):
+        gc, gs, gz = native.w4a16_quantize(W, group, sym)
+        tiled = native.w4a16_repack(gc, gs, gz, K, N, group, sym)
+        Ab, A = _acts(7, K, 5, 1)
+        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                              kernel=native.KERNEL_SKINNY)
+        assert torch.count_nonzero(C).item() == 0
+
+
+@pytest.mark.parametrize("K,N", LLAMA8B)
+def test_gemm_llama8b_decode_tiled_sampled(K, N):
+    """The four Llama-3-8B decode layers at M = 1 in the launch configuration of the benchmark
+    (tiled layout, AUTO dispatch)."""
+    group, sym, a_dtype = 128, 0, 0
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 1000 + N)
+    Ab, A = _acts(1, K, 2000 + K, a_dtype)
+    cols = synthetic.column_sample(N, 512, seed=K + N + 1)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_gemm_skinny_sweep_shape_sampled(M):
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 9000 + M, a_dtype)
+    cols = synthetic.column_sample(N, 96, seed=M + 2)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_SKINNY)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+# ----------------------------------------------------------------------------- tiled layout + CUDA-core GEMV
+GEMV_TILED = [
+    # M, K, N, group, sym, a_dtype
+    (1, 512, 256, 128, 0, 0),
+    (1, 384, 128, 128, 1, 1),     # three groups of 64 K tiles
+    (2, 768, 128, 32, 1, 1),
+    (1, 4096, 1024, 64, 0, 1),
+    (2, 2048, 384, 128, 1, 0),
+    (1, 1024, 640, 32, 0, 0),
+    (2, 4096, 256, 64, 0, 1),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", GEMV_TILED)
+def test_gemm_gemv_tiled_full_output(M, K, N, group, sym, a_dtype):
+    kind = "student_t" if sym else "normal"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 90 + K + N)
+    Ab, A = _acts(M, K, 1100 + M, a_dtype)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+def test_gemm_gemv_tiled_unit_rows(a_dtype):
+    K, N, group, sym = 512, 256, 64, 0
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
+    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
+    one = 0x3C00 if a_dtype == 0 else 0x3F80
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    for k in (0, 33, 64, 255, 511):
+        Ab = np.zeros((1, K), dtype=np.uint16)
+        Ab[0, k] = one
+        A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                              kernel=native.KERNEL_GEMV)
+        expect = oracle.decode16(oracle.encode16(What[[k]], a_dtype), a_dtype)
+        assert np.array_equal(oracle.decode16(_to_np16(C), a_dtype), expect)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemm_gemv_sweep_shape_sampled(M):
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 9500 + M, a_dtype)
+    cols = synthetic.column_sample(N, 128, seed=M + 3)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

@@ -32,6 +32,7 @@ int forced_kernel() {
         const char* e = getenv("W4A16_FORCE_KERNEL");
         if (e && strcmp(e, "gemv") == 0) forced = W4A16_KERNEL_GEMV;
         if (e && strcmp(e, "tc") == 0) forced = W4A16_KERNEL_TC;
+        if (e && strcmp(e, "skinny") == 0) forced = W4A16_KERNEL_SKINNY;
     });
     return forced;
 }
@@ -50,18 +51,18 @@ const char* kernel_name(int k) {
     switch (k) {
         case W4A16_KERNEL_GEMV: return "gemv";
         case W4A16_KERNEL_TC: return "tc";
+        case W4A16_KERNEL_SKINNY: return "skinny";
         default: return "auto";
     }
 }
 
-// The dispatch proper, without the environment override. At small M the layer is bound by the
-// weight stream and the split-K CUDA-core GEMV serves it; from M = 32 the tensor-core GEMM takes
-// over (it needs the tiled layout).
+// The dispatch proper (tiled layout), without the environment override. Up to M = 16 the layer is
+// bound by the weight stream and the split-K skinny kernel serves it; above, the tensor-core GEMM.
 int dispatch(int M, int N, int K, int group) {
     (void)N;
-    (void)K;
     (void)group;
-    return M >= 32 ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    if (M <= 2) return W4A16_KERNEL_GEMV;
+    return (M <= 16 && K % 128 == 0) ? W4A16_KERNEL_SKINNY : W4A16_KERNEL_TC;
 }
 
 }  // namespace
@@ -140,7 +141,8 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
     if (a_dtype != W4A16_F16 && a_dtype != W4A16_BF16) return W4A16_EINVAL;
     if (layout != W4A16_LAYOUT_PLAIN && layout != W4A16_LAYOUT_TILED) return W4A16_EINVAL;
     if (sym != 0 && sym != 1) return W4A16_EINVAL;
-    if (kernel != W4A16_KERNEL_AUTO && kernel != W4A16_KERNEL_GEMV && kernel != W4A16_KERNEL_TC)
+    if (kernel != W4A16_KERNEL_AUTO && kernel != W4A16_KERNEL_GEMV && kernel != W4A16_KERNEL_TC &&
+        kernel != W4A16_KERNEL_SKINNY)
         return W4A16_EINVAL;
     if (!A || !wq || !C) return W4A16_EINVAL;
     if (layout == W4A16_LAYOUT_PLAIN) {
@@ -175,8 +177,18 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
         }
         return W4A16_OK;
     }
+    if (chosen == W4A16_KERNEL_GEMV && layout == W4A16_LAYOUT_TILED) {
+        st = launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s);
+        // M > 2, or activations too long for one split's shared memory: the tensor-core kernel
+        if (st == W4A16_EUNSUPPORTED && kernel == W4A16_KERNEL_AUTO)
+            return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
+        return st;
+    }
     if (chosen == W4A16_KERNEL_TC && layout == W4A16_LAYOUT_TILED) {
         return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
+    }
+    if (chosen == W4A16_KERNEL_SKINNY && layout == W4A16_LAYOUT_TILED && M <= 16) {
+        return launch_gemm_skinny(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
     }
     return W4A16_EUNSUPPORTED;
 }

@@ -65,4 +65,10 @@ int launch_gemv_plain(const void* A, int a_dtype, int M, int K, const int32_t* c
 int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                    void* C, int* dev_status, cudaStream_t stream);
 
+int launch_gemm_skinny(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                       void* C, int* dev_status, cudaStream_t stream);
+
+int launch_gemv_tiled(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                      void* C, cudaStream_t stream);
+
 }  // namespace w4a16

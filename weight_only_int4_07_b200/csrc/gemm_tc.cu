@@ -38,7 +38,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreadsTC = 192;
+constexpr int kThreadsTC = 320;  // producer, MMA, 8 dequant/epilogue warps
 constexpr uint64_t kSpin = 2000000000ull;  // a wait gives up after 2 s (nanoseconds)
 
 template <int BN>
@@ -126,7 +126,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&afull[s], 128);
+            mbar_init(&afull[s], 256);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accfull, 1);
@@ -186,12 +186,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
                 tc_fence_after();
                 const uint32_t a_base = smem_u32(smem + s * Cfg::kStage);
                 const uint32_t b_base = a_base + Cfg::kA;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_f16_ss(tmem_d, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32),
-                               idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&empty[s]);
+                // the stage's four K-steps of 16 and the commit that frees the stage
+                mma4_f16_ss_commit(tmem_d, smem_desc_sw128(a_base), smem_desc_sw128(b_base), idesc,
+                                   it > 0 ? 1u : 0u, &empty[s]);
                 ++done;
             }
             mma_commit(accfull);  // also completes when nothing was issued
@@ -199,7 +196,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
         }
     } else {
         // ---------------------------------------------------------------- dequant + epilogue
+        // two warps per TMEM lane quarter: warp half hf dequantizes rows 4 hf .. 4 hf + 3 of the
+        // stage's code tile (K 32 hf .. 32 hf + 31) and stores columns [BN/2 hf, BN/2 (hf + 1)) of C
         const int q = warp & 3;           // tensor-memory lane quarter this warp may access
+        const int hf = (warp - 2) >> 2;   // 0 for warps 2..5, 1 for warps 6..9
         const int n = 32 * q + lane;      // output channel within the tile = TMEM lane
         Deq<T> dq;
         bool ok = true;
@@ -214,19 +214,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
             const __half* ssm = reinterpret_cast<const __half*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes);
             const uint32_t* zsm = reinterpret_cast<const uint32_t*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales);
             uint8_t* atile = st;
-            const uint4 wlo = ctile[n];          // words of rows 0..3 of the stage (half 0)
-            const uint4 whi = ctile[128 + n];    // rows 4..7 (half 1)
-            const uint32_t words[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
-            const int rows_per_group = group / 8;
+            const uint4 w4 = ctile[128 * hf + n];   // rows 4 hf .. 4 hf + 3 of the stage
+            const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+            // group of this half inside the stage (group 32: one group per half)
+            const int lg = groups_per_stage > 1 ? hf : 0;
+            const float sv = __half2float(ssm[lg * 128 + n]);
+            const int zv = sym ? 8 : (int)((zsm[lg * 16 + n / 8] >> (4 * (n % 8))) & 0xFu);
+            dq.set(sv, zv);
 #pragma unroll
-            for (int jl = 0; jl < 8; ++jl) {
-                if (jl == 0 || (groups_per_stage > 1 && jl % rows_per_group == 0)) {
-                    const int lg = groups_per_stage > 1 ? jl / rows_per_group : 0;
-                    const float sv = __half2float(ssm[lg * 128 + n]);
-                    const int zv = sym ? 8 : (int)((zsm[lg * 16 + n / 8] >> (4 * (n % 8))) & 0xFu);
-                    dq.set(sv, zv);
-                }
-                const uint32_t w = words[jl];
+            for (int i = 0; i < 4; ++i) {
+                const int jl = 4 * hf + i;
+                const uint32_t w = words[i];
                 uint4 out;
                 out.x = dq.pair((w & 0x000F000Fu) | Deq<T>::kMagic);
                 out.y = dq.pair(((w >> 4) & 0x000F000Fu) | Deq<T>::kMagic);
@@ -239,12 +237,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
             fence_proxy_async_smem();
             mbar_arrive(&afull[s]);
         }
-        // epilogue: D (lane n, columns 0..BN-1) -> C[m0 + m, n0 + n]
+        // epilogue: D (lane n, columns 0..BN-1) -> C[m0 + m, n0 + n]; this warp stores half the columns
         if (mbar_wait(accfull, 0, abort_flag, dev_status, kSpin) && ok && !*abort_flag) {
             tc_fence_after();
             const uint32_t lane_base = tmem_d + ((uint32_t)(32 * q) << 16);
+            constexpr int kChunks = BN / 16;
+            const int c0 = kChunks > 1 ? hf * (kChunks / 2) : 0;
+            const int c1 = kChunks > 1 ? c0 + kChunks / 2 : (hf == 0 ? 1 : 0);
 #pragma unroll 1
-            for (int c = 0; c < BN / 16; ++c) {
+            for (int c = c0; c < c1; ++c) {
                 uint32_t v[16];
                 tmem_ld16(lane_base + c * 16, v);
                 tmem_ld_wait();
@@ -265,8 +266,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
     }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -294,6 +297,8 @@ bool make_act_map(CUtensorMap* map, const void* A, int M, int K, int box_rows, b
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int BN, typename T>
 int launch_tc_typed(const void* A, int M, int K, const void* tiled, int N, int group, int sym, void* C,
