@@ -83,7 +83,7 @@ def test_select_kernel_and_workspace_are_host_only(L):
         assert k in (native.KERNEL_GEMV, native.KERNEL_TC, native.KERNEL_SKINNY)
         # decode-sized M streams the weights (GEMV, then the skinny split-K kernel); larger M uses
         # the tensor-core GEMM
-        assert k == (native.KERNEL_GEMV if M <= 2 else native.KERNEL_SKINNY if M <= 16 else native.KERNEL_TC)
+        assert k == (native.KERNEL_GEMV if M <= 16 else native.KERNEL_TC)
         assert native.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
     assert native.w4a16_workspace_bytes(0, 4096, 4096, 128) == 0
     assert native.w4a16_workspace_bytes(1, 4096, 4000, 128) == 0

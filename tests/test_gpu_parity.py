@@ -478,3 +478,27 @@ def test_gemm_gemv_sweep_shape_sampled(M):
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SKINNY_GEMM)
+def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype):
+    """The decode kernel (warp-level MMA) at M = 1..16 on the tiled layout."""
+    kind = "student_t" if sym else "normal"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 70 + K + N)
+    Ab, A = _acts(M, K, 1300 + M, a_dtype)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+
+
+@pytest.mark.parametrize("M", [4, 9, 16])
+def test_gemm_gemv_mma_sweep_shape_sampled(M):
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 9700 + M, a_dtype)
+    cols = synthetic.column_sample(N, 96, seed=M + 4)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

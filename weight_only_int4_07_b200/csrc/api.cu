@@ -61,8 +61,7 @@ const char* kernel_name(int k) {
 int dispatch(int M, int N, int K, int group) {
     (void)N;
     (void)group;
-    if (M <= 2) return W4A16_KERNEL_GEMV;
-    return (M <= 16 && K % 128 == 0) ? W4A16_KERNEL_SKINNY : W4A16_KERNEL_TC;
+    return (M <= 16 && K % 128 == 0) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_TC;
 }
 
 }  // namespace
@@ -178,7 +177,9 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
         return W4A16_OK;
     }
     if (chosen == W4A16_KERNEL_GEMV && layout == W4A16_LAYOUT_TILED) {
-        st = launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s);
+        st = (getenv("W4A16_GEMV_CUDA_CORES") != nullptr)
+                 ? launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s)
+                 : launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
         // M > 2, or activations too long for one split's shared memory: the tensor-core kernel
         if (st == W4A16_EUNSUPPORTED && kernel == W4A16_KERNEL_AUTO)
             return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);

@@ -71,4 +71,7 @@ int launch_gemm_skinny(const void* A, int a_dtype, int M, int K, const void* til
 int launch_gemv_tiled(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                       void* C, cudaStream_t stream);
 
+int launch_gemv_mma(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                    void* C, cudaStream_t stream);
+
 }  // namespace w4a16
