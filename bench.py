@@ -198,7 +198,7 @@ class DecodeStack:
         self.C = torch.empty(self.c_elems, dtype=torch.float16, device=dev)
         self.C_host = torch.empty(self.c_elems, dtype=torch.float16).pin_memory()
         ws = max(native.w4a16_workspace_bytes(M, N, K, GROUP) for (_, K, N) in LLAMA8B_LINEARS)
-        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        self.ws = torch.zeros(max(ws, 16), dtype=torch.uint8, device=dev)
         # views per GEMM
         self.calls = []
         ao = co = 0
@@ -344,7 +344,7 @@ def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
     del W
     use_tiled = tiled_supported(torch, native, (K, N, codes, scales, zeros), M)
     ws_need = native.w4a16_workspace_bytes(M, N, K, GROUP)
-    ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(ws_need, 16), dtype=torch.uint8, device=dev)
     if use_tiled:
         mats = [(None, None, None, native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM))
                 for _ in range(copies)]

@@ -141,18 +141,24 @@ W4A16_API int w4a16_repack(const int32_t* codes, const void* scales, const int32
                  int group, int sym, void* tiled, void* stream);
 
 /*
- * w4a16_workspace_bytes -- device scratch that w4a16_gemm needs for an M x N x K call with the
- * kernel the dispatch picks (split-K partial sums and their counters). 0 when none is needed.
+ * w4a16_workspace_bytes -- device scratch that w4a16_gemm needs for an M x N x K call, large
+ * enough for any kernel the call may run: 64 KiB of per-tile counters of the stream-K decode
+ * kernel, followed by split-K FP32 partial sums. Depends on the SM count of the current device.
+ * Returns 0 only for arguments w4a16_gemm rejects.
  */
 W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
 
 /*
  * w4a16_select_kernel -- the M-based dispatch, as a pure host function: returns the
  * w4a16_kernel that w4a16_gemm(..., W4A16_KERNEL_AUTO) runs on the tiled layout for this shape.
- * Small M is bound by the weight stream and goes to the split-K skinny kernel; larger M goes to
- * the tensor-core GEMM ("INT8 vs INT4 Quantization, in depth", section "Two regimes: waiting for
- * memory, waiting for math"). The plain layout always runs the CUDA-core GEMV.
+ * M <= 16 is bound by the weight stream and goes to the decode GEMV (W4A16_KERNEL_GEMV); larger M
+ * goes to the tensor-core GEMM ("INT8 vs INT4 Quantization, in depth", section "Two regimes:
+ * waiting for memory, waiting for math"). The plain layout always runs the CUDA-core GEMV.
  * The environment variable W4A16_FORCE_KERNEL=gemv|tc|skinny overrides the choice.
+ * On the tiled layout the decode GEMV is the persistent stream-K kernel (one CTA per SM, bulk-copy
+ * pipeline, warp-level tensor-core MMA); when M rows of A do not fit in its shared memory it runs
+ * the cluster split-K variant. W4A16_GEMV_VARIANT=cluster|cuda_cores forces the cluster variant
+ * or the CUDA-core variant (M <= 2).
  */
 W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
 
@@ -171,12 +177,17 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
  *   N, group   output channels; group size.
  *   sym        1 = symmetric codes, 0 = asymmetric (must match how the weight was quantized).
  *   C          device out, [M, N] row-major, dtype a_dtype. Must not alias A or the weights.
- *   workspace  device scratch of at least w4a16_workspace_bytes(M, N, K, group) bytes (NULL if 0).
- *              Calls that share one workspace must be ordered on the GPU (same stream).
+ *   workspace  device scratch of at least w4a16_workspace_bytes(M, N, K, group) bytes, 16-byte
+ *              aligned, owned by the caller. Its first 64 KiB (tile counters) must be zero before
+ *              the first call that uses it; every call that completes without a device error
+ *              leaves them zero, so a workspace is zeroed once, at allocation. Calls that share
+ *              one workspace must be ordered on the GPU (same stream). After a call that set
+ *              dev_status to W4A16_ETIMEOUT, zero the workspace again.
  *   ws_bytes   size of workspace.
  *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC /
- *              W4A16_KERNEL_SKINNY. GEMV reads the PLAIN layout only; TC and SKINNY read the TILED
- *              layout only; SKINNY needs M <= 16. Other combinations return W4A16_EUNSUPPORTED.
+ *              W4A16_KERNEL_SKINNY. GEMV reads both layouts (TILED: M <= 16, K % 128 == 0); TC and
+ *              SKINNY read the TILED layout only; SKINNY needs M <= 16. Other combinations return
+ *              W4A16_EUNSUPPORTED.
  *   dev_status device int or NULL: set to W4A16_ETIMEOUT if a bounded on-device wait gave up
  *              (the output is then unspecified; the device stays usable).
  *   stream     cudaStream_t.

@@ -441,8 +441,13 @@ GEMV_TILED = [
 ]
 
 
+@pytest.fixture
+def cuda_cores(monkeypatch):
+    monkeypatch.setenv("W4A16_GEMV_VARIANT", "cuda_cores")
+
+
 @pytest.mark.parametrize("M,K,N,group,sym,a_dtype", GEMV_TILED)
-def test_gemm_gemv_tiled_full_output(M, K, N, group, sym, a_dtype):
+def test_gemm_gemv_tiled_full_output(M, K, N, group, sym, a_dtype, cuda_cores):
     kind = "student_t" if sym else "normal"
     Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 90 + K + N)
     Ab, A = _acts(M, K, 1100 + M, a_dtype)
@@ -453,7 +458,7 @@ def test_gemm_gemv_tiled_full_output(M, K, N, group, sym, a_dtype):
 
 
 @pytest.mark.parametrize("a_dtype", [0, 1])
-def test_gemm_gemv_tiled_unit_rows(a_dtype):
+def test_gemm_gemv_tiled_unit_rows(a_dtype, cuda_cores):
     K, N, group, sym = 512, 256, 64, 0
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
     What = oracle.dequant(oc, os_, oz, K, N, group, sym)
@@ -470,19 +475,30 @@ def test_gemm_gemv_tiled_unit_rows(a_dtype):
 
 
 @pytest.mark.parametrize("M", [1, 2])
-def test_gemm_gemv_sweep_shape_sampled(M):
+def test_gemm_gemv_sweep_shape_sampled(M, cuda_cores):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9500 + M, a_dtype)
     cols = synthetic.column_sample(N, 128, seed=M + 3)
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
 
 
+@pytest.fixture(params=["stream", "cluster"])
+def mma_variant(request, monkeypatch):
+    if request.param == "cluster":
+        monkeypatch.setenv("W4A16_GEMV_VARIANT", "cluster")
+    else:
+        monkeypatch.delenv("W4A16_GEMV_VARIANT", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SKINNY_GEMM)
-def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype):
-    """The decode kernel (warp-level MMA) at M = 1..16 on the tiled layout."""
+def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype, mma_variant):
+    """The decode kernels (warp-level MMA: persistent stream-K and cluster split-K) at M = 1..16
+    on the tiled layout."""
     kind = "student_t" if sym else "normal"
     Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 70 + K + N)
     Ab, A = _acts(M, K, 1300 + M, a_dtype)
@@ -493,12 +509,102 @@ def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype):
 
 
 @pytest.mark.parametrize("M", [4, 9, 16])
-def test_gemm_gemv_mma_sweep_shape_sampled(M):
+def test_gemm_gemv_mma_sweep_shape_sampled(M, mma_variant):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9700 + M, a_dtype)
     cols = synthetic.column_sample(N, 96, seed=M + 4)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
                           kernel=native.KERNEL_GEMV)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+# ----------------------------------------------------------------------------- stream-K decode GEMV
+STREAM_GEMM = [
+    # M, K, N, group, sym, a_dtype      (units = N/128 * K/128 against one CTA per SM)
+    (1, 128, 128, 128, 0, 0),           # one unit, one CTA
+    (1, 8192, 128, 128, 0, 1),          # one tile cut among 64 CTAs
+    (3, 16384, 256, 128, 1, 0),         # two tiles, each cut among about 74 CTAs
+    (1, 4096, 1024, 32, 0, 0),          # 256 units: tiles cut in two
+    (8, 2048, 1280, 64, 1, 1),
+    (9, 1024, 2560, 128, 0, 1),         # two n8 tiles of rows
+    (16, 3072, 768, 32, 1, 0),
+    (1, 14336, 512, 128, 1, 1),         # long K, symmetric reference chains
+    (2, 4096, 6144, 128, 0, 0),         # every CTA holds whole tiles and cut ones
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", STREAM_GEMM)
+def test_gemm_stream_full_output(M, K, N, group, sym, a_dtype):
+    kind = "student_t" if sym else "outliers"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 110 + K + N)
+    Ab, A = _acts(M, K, 1500 + M, a_dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+    # the tile counters are back at zero, and a second call on the same workspace is identical
+    assert torch.count_nonzero(ws[:65536]).item() == 0
+    C2 = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                           kernel=native.KERNEL_GEMV, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(C.view(torch.int16), C2.view(torch.int16))
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+@pytest.mark.parametrize("sym", [0, 1])
+@pytest.mark.parametrize("group", [128, 32])
+def test_gemm_stream_unit_rows_return_dequantized_rows(a_dtype, sym, group):
+    """A = unit rows: each output row is one dequantized weight row rounded once, bit for bit,
+    also through the reference-chain correction of group 128."""
+    K, N = 1024, 384
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 41)
+    rows = [0, 1, 2, 3, 8, 9, 31, 32, 63, 64, 127, 128, 500, 777, 1022, 1023]
+    Ab = np.zeros((len(rows), K), dtype=np.uint16)
+    one = 0x3C00 if a_dtype == 0 else 0x3F80
+    for i, k in enumerate(rows):
+        Ab[i, k] = one
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
+    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
+    expect = oracle.decode16(oracle.encode16(What[rows], a_dtype), a_dtype)
+    for m in (1, 5, 16):
+        C = native.w4a16_gemm(A[:m].contiguous(), tiled, None, None, N, group, sym,
+                              layout=native.LAYOUT_TILED, kernel=native.KERNEL_GEMV)
+        assert np.array_equal(oracle.decode16(_to_np16(C), a_dtype), expect[:m])
+
+
+@pytest.mark.parametrize("a_dtype", [0, 1])
+def test_gemm_stream_zero_weights_give_exact_zero(a_dtype):
+    """All-zero weight columns give exactly zero (the bound there is 1e-5 absolute), for the
+    asymmetric (code 0, zero 0) and symmetric (offset-binary 8) references."""
+    K, N = 2048, 512
+    W = torch.zeros((K, N), dtype=torch.float16, device="cuda")
+    W[:, 256:] = torch.from_numpy(synthetic.weights_normal(K, 256, seed=3).view(np.int16)).view(
+        torch.float16).cuda()
+    for sym in (0, 1):
+        for group in (128, 64):
+            gc, gs, gz = native.w4a16_quantize(W, group, sym)
+            tiled = native.w4a16_repack(gc, gs, gz, K, N, group, sym)
+            for M in (1, 11):
+                Ab, A = _acts(M, K, 7 + M, a_dtype)
+                C = native.w4a16_gemm(A, tiled, None, None, N, group, sym,
+                                      layout=native.LAYOUT_TILED, kernel=native.KERNEL_GEMV)
+                assert torch.count_nonzero(C[:, :256]).item() == 0
+                assert torch.count_nonzero(C[:, 256:]).item() > 0
+
+
+@pytest.mark.parametrize("K,N", [(8192, 10240), (8192, 8192), (8192, 57344), (28672, 8192)])
+def test_gemm_stream_llama70b_decode_sampled(K, N):
+    """The Llama-3-70B-shaped layers at M = 1 (bf16), sampled columns."""
+    group, sym, a_dtype = 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 3000 + N)
+    Ab, A = _acts(1, K, 4000 + K, a_dtype)
+    cols = synthetic.column_sample(N, 256, seed=K + N + 7)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

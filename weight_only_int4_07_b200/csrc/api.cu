@@ -125,9 +125,14 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group) {
 
 W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group) {
     if (M < 1 || check_shape(K, N, group) != W4A16_OK) return 0;
-    // the largest need over every kernel a call may run, so a forced kernel also fits
+    // the largest need over every kernel a call may run, so a forced kernel also fits; the tile
+    // counters of the stream-K kernel come first and are always reserved
     const GemvPlan p = plan_gemv_plain(M, N, K, group);
-    return p.ws_bytes;
+    int n_sm = gemv_stream_sm_count();
+    if (n_sm <= 0) n_sm = 148;
+    const GemvStreamPlan q = plan_gemv_stream(M, N, K, group, n_sm);
+    const size_t rest = q.ok && q.partial_bytes > p.ws_bytes ? q.partial_bytes : p.ws_bytes;
+    return kGemvStreamCounterBytes + rest;
 }
 
 W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* wq, int layout,
@@ -155,6 +160,8 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
     const size_t need = w4a16_workspace_bytes(M, N, K, group);
     if (ws_bytes < need || (need > 0 && !workspace)) return W4A16_EWORKSPACE;
     if (workspace && !aligned16(workspace)) return W4A16_EALIGN;
+    // partial sums of the split-K kernels live after the stream-K tile counters
+    void* scratch = static_cast<char*>(workspace) + kGemvStreamCounterBytes;
 
     int chosen = kernel == W4A16_KERNEL_AUTO ? w4a16_select_kernel(M, N, K, group) : kernel;
     // the plain layout has only the CUDA-core kernel
@@ -171,16 +178,23 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
             const int mc = (M - m0) < p.mt ? (M - m0) : p.mt;
             st = launch_gemv_plain(static_cast<const char*>(A) + (size_t)m0 * K * elt, a_dtype, mc, K,
                                    static_cast<const int32_t*>(wq), scales, zeros, N, group, sym,
-                                   static_cast<char*>(C) + (size_t)m0 * N * elt, workspace, p, s);
+                                   static_cast<char*>(C) + (size_t)m0 * N * elt, scratch, p, s);
             if (st != W4A16_OK) return st;
         }
         return W4A16_OK;
     }
     if (chosen == W4A16_KERNEL_GEMV && layout == W4A16_LAYOUT_TILED) {
-        st = (getenv("W4A16_GEMV_CUDA_CORES") != nullptr)
-                 ? launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s)
-                 : launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
-        // M > 2, or activations too long for one split's shared memory: the tensor-core kernel
+        const char* variant = getenv("W4A16_GEMV_VARIANT");
+        if (variant && strcmp(variant, "cuda_cores") == 0) {
+            st = launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s);
+        } else if (variant && strcmp(variant, "cluster") == 0) {
+            st = launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
+        } else {
+            st = launch_gemv_stream(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
+            // activations of M rows too long for shared memory: the cluster split-K kernel
+            if (st == W4A16_EUNSUPPORTED) st = launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
+        }
+        // M > 16, or activations too long for one split's shared memory: the tensor-core kernel
         if (st == W4A16_EUNSUPPORTED && kernel == W4A16_KERNEL_AUTO)
             return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
         return st;

@@ -74,4 +74,21 @@ int launch_gemv_tiled(const void* A, int a_dtype, int M, int K, const void* tile
 int launch_gemv_mma(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                     void* C, cudaStream_t stream);
 
+// Persistent stream-K decode kernel. Its workspace starts with one int counter per 128-channel
+// tile (kGemvStreamCounterBytes, zero between calls; each call leaves them zero), followed by
+// the FP32 partial sums of tiles cut between CTAs.
+constexpr size_t kGemvStreamCounterBytes = 64 * 1024;
+constexpr int kGemvStreamMaxTiles = (int)(kGemvStreamCounterBytes / 4);
+struct GemvStreamPlan {
+    bool ok;
+    int ns;               // pipeline stages
+    int ctas;             // persistent CTAs (one per SM)
+    size_t act_bytes, ref_bytes, red_bytes, smem;
+    size_t partial_bytes; // workspace after the counters
+};
+GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int n_sm);
+int gemv_stream_sm_count();
+int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                       void* C, void* workspace, int* dev_status, cudaStream_t stream);
+
 }  // namespace w4a16

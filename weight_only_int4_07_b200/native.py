@@ -147,7 +147,8 @@ def w4a16_gemm(A, wq, scales, zeros, N, group, sym, layout=LAYOUT_PLAIN, C=None,
         C = torch.empty((M, N), dtype=A.dtype, device=A.device)
     need = w4a16_workspace_bytes(M, N, K, group)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
+        # the tile counters at the front of a workspace must start at zero
+        workspace = torch.zeros(need, dtype=torch.uint8, device=A.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().w4a16_gemm(_ptr(A), a_dtype, M, K, _ptr(wq), int(layout), _ptr(scales), _ptr(zeros),
                           N, group, int(sym), _ptr(C), _ptr(workspace), ws_bytes, int(kernel),
