@@ -77,10 +77,9 @@ typedef enum {
 /* Kernel family chosen by the M-based dispatch (see w4a16_select_kernel). */
 typedef enum {
     W4A16_KERNEL_AUTO = 0,    /* let the dispatch decide                                      */
-    W4A16_KERNEL_GEMV = 1,    /* split-K CUDA-core GEMV (plain layout), any M                 */
-    W4A16_KERNEL_TC = 2,      /* tcgen05 tensor-core GEMM, TMEM accumulator (tiled layout)     */
-    W4A16_KERNEL_SKINNY = 3   /* split-K tcgen05 kernel for M <= 16, exact integer weights in
-                                 TMEM, per-group FP32 scaling, cluster reduction (tiled layout) */
+    W4A16_KERNEL_GEMV = 1,    /* decode GEMV: split-K CUDA-core (plain layout, any M) or the
+                                 persistent stream-K warp-MMA kernel (tiled layout, M <= 16) */
+    W4A16_KERNEL_TC = 2       /* tcgen05 tensor-core GEMM, TMEM accumulator (tiled layout)     */
 } w4a16_kernel;
 
 /*
@@ -121,19 +120,22 @@ W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);
  * re-quantized. "INT4 and Low-Bit Inference", section 5 "The kernel is half the story" (weights
  * pre-permuted at load so unpacking is branch-free and coalesced); "4.3 Weight-only INT4",
  * section 4 (weights pre-reordered into a layout that suits runtime reads).
- * Tiled layout: the weight is cut into tiles of 128 output channels x 64 input channels
- * (tile (t, c) covers n in [128 t, 128 t + 128), k in [64 c, 64 c + 64)). Tiles are stored in
- * order c-major-within-t: tile index = t * (K / 64) + c; each tile is 128 x 8 = 1024 int32 words
- * (4 KiB) holding word (j, n) of the plain layout at offset
- *     ((j % 8) / 4) * 512 + (n % 128) * 4 + (j % 4)            (j = 8 c + j % 8)
- * so that one 16-byte vector holds four consecutive words along K of one output channel, and a
- * warp's 32 consecutive output channels read 512 contiguous bytes. Each word is re-encoded:
- * nibble slot p (bits 4p..4p+3, p = 0..3) holds the code of element 2p (k = 8j + 2p) and slot
- * p + 4 that of element 2p + 1; symmetric codes are stored offset-binary, q + 8, so that both
- * schemes dequantize as (u - z) * s with z = 8 for the symmetric one. Scales and zeros follow the
- * codes in the same buffer, in the plain layouts [K/g, N] fp16 and [K/g, N/8] int32 (asym),
- * each starting on a 256-byte boundary.
- * Requires N % 128 == 0 and K % 64 == 0 (else W4A16_EUNSUPPORTED).
+ * Tiled layout: one record per unit of 128 output channels x 128 input channels; unit (t, c)
+ * covers n in [128 t, 128 t + 128), k in [128 c, 128 c + 128) and has record index
+ * t * (K / 128) + c. Records follow each other with no padding; a record is
+ *     R = 8192 + G * 256 + (sym ? 0 : G * 64) bytes,  G = 128 / group:
+ *   bytes [0, 8192)   codes: block h (h = 0..3, k in [128 c + 32 h, + 32)) at 2048 h; channel
+ *                     n % 128 owns the 16 bytes at slot ((n % 128) XOR 2h) of its block, and word
+ *                     w (w = 0..3) of them is plain word (j, n) with j = 16 c + 4 h + w;
+ *   then G x 256 B    scales: group row c * G + gg at 256 gg, channel n % 128 at + 2 (n % 128);
+ *   then G x 64 B     zeros (asym only): group row c * G + gg at 64 gg, plain words
+ *                     [16 t, 16 t + 16) of that row.
+ * Each word is re-encoded: nibble slot p (bits 4p..4p+3, p = 0..3) holds the code of element 2p
+ * (k = 8j + 2p) and slot p + 4 that of element 2p + 1; symmetric codes are stored offset-binary,
+ * q + 8, so that both schemes dequantize as (u - z) * s with z = 8 for the symmetric one.
+ * A range of consecutive units is one contiguous range of bytes (one bulk copy), and the XOR slot
+ * keeps the warp-level MMA's 16-byte reads of four blocks of one channel on different banks.
+ * Requires N % 128 == 0 and K % 128 == 0 (else W4A16_EUNSUPPORTED).
  * Arguments: codes, scales, zeros as produced by w4a16_quantize (zeros NULL iff sym);
  * tiled = device out of w4a16_repack_bytes() bytes; stream.
  */
@@ -154,11 +156,10 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
  * M <= 16 is bound by the weight stream and goes to the decode GEMV (W4A16_KERNEL_GEMV); larger M
  * goes to the tensor-core GEMM ("INT8 vs INT4 Quantization, in depth", section "Two regimes:
  * waiting for memory, waiting for math"). The plain layout always runs the CUDA-core GEMV.
- * The environment variable W4A16_FORCE_KERNEL=gemv|tc|skinny overrides the choice.
- * On the tiled layout the decode GEMV is the persistent stream-K kernel (one CTA per SM, bulk-copy
- * pipeline, warp-level tensor-core MMA); when M rows of A do not fit in its shared memory it runs
- * the cluster split-K variant. W4A16_GEMV_VARIANT=cluster|cuda_cores forces the cluster variant
- * or the CUDA-core variant (M <= 2).
+ * The environment variable W4A16_FORCE_KERNEL=gemv|tc overrides the choice.
+ * On the tiled layout the decode GEMV is the persistent stream-K kernel (one CTA per SM, unit
+ * records streamed by bulk copies, warp-level tensor-core MMA). When M rows of A do not fit in
+ * its shared memory, W4A16_KERNEL_AUTO runs the tensor-core GEMM instead.
  */
 W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
 
@@ -184,10 +185,9 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
  *              one workspace must be ordered on the GPU (same stream). After a call that set
  *              dev_status to W4A16_ETIMEOUT, zero the workspace again.
  *   ws_bytes   size of workspace.
- *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC /
- *              W4A16_KERNEL_SKINNY. GEMV reads both layouts (TILED: M <= 16, K % 128 == 0); TC and
- *              SKINNY read the TILED layout only; SKINNY needs M <= 16. Other combinations return
- *              W4A16_EUNSUPPORTED.
+ *   kernel     W4A16_KERNEL_AUTO, or a forced W4A16_KERNEL_GEMV / W4A16_KERNEL_TC. GEMV reads both
+ *              layouts (TILED: M <= 16); TC reads the TILED layout only. Other combinations
+ *              return W4A16_EUNSUPPORTED.
  *   dev_status device int or NULL: set to W4A16_ETIMEOUT if a bounded on-device wait gave up
  *              (the output is then unspecified; the device stays usable).
  *   stream     cudaStream_t.

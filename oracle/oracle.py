@@ -186,10 +186,11 @@ def within_bound(y, y_ref, y_abs, rel=2e-3, abs_=1e-5):
 
 # ----------------------------------------------------------------------------- tiled layout
 def tiled_offsets(K, N, group, sym):
-    """dict of byte offsets/sizes of the tiled buffer's regions and its total size."""
+    """Sizes of the tiled buffer: bytes per unit record, the codes / scales / zeros offsets and
+    sizes inside a record, and the whole buffer's size."""
     out = np.zeros(7, dtype=np.int64)
     _load().w4o_tiled_offsets(K, N, group, int(sym), _ptr(out))
-    keys = ("codes", "codes_bytes", "scales", "scales_bytes", "zeros", "zeros_bytes", "total")
+    keys = ("record", "codes_bytes", "scales", "scales_bytes", "zeros", "zeros_bytes", "total")
     return {k: int(v) for k, v in zip(keys, out)}
 
 

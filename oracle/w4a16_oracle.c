@@ -325,60 +325,70 @@ int w4o_max_threads(void) {
 }
 
 /* ---------------------------------------------------------------------------------------------
- * The tiled weight buffer of the library's repack entry point, restated from its definition:
- * tiles of 128 output channels x 64 input channels (8 packed rows); tile (t, c) has index
- * t * (K/64) + c and holds 1024 words; plain word (j, n) sits at
- *   ((j mod 8) div 4) * 512 + (n mod 128) * 4 + (j mod 4)
- * inside its tile, with its codes re-ordered: nibble slot p (p = 0..3) holds the code of element
- * 2p and slot p + 4 that of element 2p + 1 (element e = row k - 8j of the word); symmetric codes
- * are stored offset-binary, q + 8 (zero-point 8).
- * Scales (plain [K/g, N] fp16) and zeros (plain [K/g, N/8] int32, asym only)
- * follow, each region starting at a multiple of 256 bytes. Padding bytes are left zero.
- * (The pages ask for a pre-permuted layout -- "INT4 and Low-Bit Inference", section 5
- * "The kernel is half the story" -- but leave its form open; this one is the library's.)
+ * The tiled weight buffer of the library's repack entry point, restated from its definition.
+ * The pages ask for weights permuted once at load into a layout that suits the kernel
+ * ("INT4 and Low-Bit Inference", section 5 "The kernel is half the story"; "4.3 Weight-only
+ * INT4", section 4) and leave its form open; this is the library's.
+ *
+ * Unit (t, c) = output channels [128 t, 128 t + 128) x input channels [128 c, 128 c + 128); its
+ * record has index t * (K/128) + c and R = 8192 + G * 256 + (asym ? G * 64 : 0) bytes, where
+ * G = 128 / group groups of K fall in a unit. Inside a record:
+ *   codes, bytes [0, 8192): block h (h = 0..3, input channels 128 c + 32 h .. + 31) at 2048 h;
+ *     in it, channel n (n = 0..127 within the tile) owns the 16 bytes at slot (n XOR 2 h); word
+ *     w (w = 0..3) of those 16 bytes is plain packed row j = 16 c + 4 h + w of channel 128 t + n,
+ *     its codes re-ordered: nibble slot p (p = 0..3) holds the code of element 2p and slot p + 4
+ *     that of element 2p + 1 (element e = input channel 8 j + e); symmetric codes are stored
+ *     offset-binary, q + 8 (zero-point 8);
+ *   scales, from byte 8192: group gg (gg = 0..G-1, plain group row c * G + gg) at 8192 + 256 gg,
+ *     channel n at + 2 n (fp16 bits);
+ *   zeros (asymmetric only), from byte 8192 + 256 G: group gg at + 64 gg, the 16 plain words of
+ *     the tile's channels (word n / 8 holds channel n at nibble n mod 8).
+ * Records follow each other with no padding.
  * ------------------------------------------------------------------------------------------- */
-static long round_up_256(long x) { return (x + 255) / 256 * 256; }
-
 void w4o_tiled_offsets(long K, long N, long group, int sym, long* out) {
-    const long codes_bytes = K * N / 2;
-    const long scales_off = round_up_256(codes_bytes);
-    const long scales_bytes = (K / group) * N * 2;
-    const long zeros_off = round_up_256(scales_off + scales_bytes);
-    const long zeros_bytes = sym ? 0 : (K / group) * (N / 8) * 4;
-    out[0] = 0;
-    out[1] = codes_bytes;
-    out[2] = scales_off;
-    out[3] = scales_bytes;
-    out[4] = zeros_off;
-    out[5] = zeros_bytes;
-    out[6] = round_up_256(zeros_off + zeros_bytes);
+    const long G = 128 / group;
+    const long record = 8192 + G * 256 + (sym ? 0 : G * 64);
+    out[0] = record;                 /* bytes per unit record */
+    out[1] = 8192;                   /* codes bytes per record */
+    out[2] = 8192;                   /* scales offset in a record */
+    out[3] = G * 256;                /* scales bytes per record */
+    out[4] = 8192 + G * 256;         /* zeros offset in a record */
+    out[5] = sym ? 0 : G * 64;       /* zeros bytes per record */
+    out[6] = (N / 128) * (K / 128) * record;   /* whole buffer */
 }
 
 int w4o_repack(const int32_t* codes, const uint16_t* scales, const int32_t* zeros, long K, long N,
                long group, int sym, uint8_t* out) {
-    if (!valid_shape(K, N, group) || N % 128 != 0 || K % 64 != 0) return W4O_EINVAL;
+    if (!valid_shape(K, N, group) || N % 128 != 0 || K % 128 != 0) return W4O_EINVAL;
     long off[7];
     w4o_tiled_offsets(K, N, group, sym, off);
+    const long R = off[0], G = 128 / group, units = K / 128;
     memset(out, 0, (size_t)off[6]);
-    int32_t* tiled = (int32_t*)out;
-    const long ktiles = K / 64;
     for (long t = 0; t < N / 128; ++t)
-        for (long c = 0; c < ktiles; ++c)
-            for (long jl = 0; jl < 8; ++jl)
-                for (long nl = 0; nl < 128; ++nl) {
-                    const long j = 8 * c + jl, n = 128 * t + nl;
-                    const long pos = (t * ktiles + c) * 1024 + (jl / 4) * 512 + nl * 4 + (jl % 4);
-                    const uint32_t w = (uint32_t)codes[j * N + n];
-                    uint32_t t = 0;
-                    for (int e = 0; e < 8; ++e) {
-                        uint32_t u = (w >> (4 * e)) & 0xFu;            /* element e */
-                        if (sym) u = (u + 8u) & 0xFu;                  /* q + 8 for q in -8..7 */
-                        const int slot = (e % 2 == 0) ? e / 2 : 4 + e / 2;
-                        t |= u << (4 * slot);
+        for (long c = 0; c < units; ++c) {
+            uint8_t* rec = out + (t * units + c) * R;
+            for (long h = 0; h < 4; ++h)
+                for (long nl = 0; nl < 128; ++nl)
+                    for (long w = 0; w < 4; ++w) {
+                        const long j = 16 * c + 4 * h + w, n = 128 * t + nl;
+                        const uint32_t word = (uint32_t)codes[j * N + n];
+                        uint32_t enc = 0;
+                        for (int e = 0; e < 8; ++e) {
+                            uint32_t u = (word >> (4 * e)) & 0xFu;     /* element e */
+                            if (sym) u = (u + 8u) & 0xFu;              /* q + 8 for q in -8..7 */
+                            const int slot = (e % 2 == 0) ? e / 2 : 4 + e / 2;
+                            enc |= u << (4 * slot);
+                        }
+                        memcpy(rec + 2048 * h + 16 * (nl ^ (2 * h)) + 4 * w, &enc, 4);
                     }
-                    tiled[pos] = (int32_t)t;
-                }
-    memcpy(out + off[2], scales, (size_t)off[3]);
-    if (!sym) memcpy(out + off[4], zeros, (size_t)off[5]);
+            for (long gg = 0; gg < G; ++gg) {
+                const long gi = c * G + gg;
+                for (long nl = 0; nl < 128; ++nl)
+                    memcpy(rec + off[2] + 256 * gg + 2 * nl, &scales[gi * N + 128 * t + nl], 2);
+                if (!sym)
+                    for (long wd = 0; wd < 16; ++wd)
+                        memcpy(rec + off[4] + 64 * gg + 4 * wd, &zeros[gi * (N / 8) + 16 * t + wd], 4);
+            }
+        }
     return W4O_OK;
 }

@@ -64,25 +64,24 @@ def test_status_strings(L):
 
 
 def test_repack_bytes(L):
-    # codes K*N/2, then scales (K/g)*N*2 and zeros (K/g)*(N/8)*4, each on a 256-byte boundary
-    K, N, g = 4096, 4096, 128
-    codes = K * N // 2
-    scales = (K // g) * N * 2
-    zeros = (K // g) * (N // 8) * 4
-    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert native.w4a16_repack_bytes(K, N, g, 0) == up(up(up(codes) + scales) + zeros)
-    assert native.w4a16_repack_bytes(K, N, g, 1) == up(up(codes) + scales)
-    assert native.w4a16_repack_bytes(K, 8, g, 0) == 0          # N not a multiple of 128
-    assert native.w4a16_repack_bytes(96, 128, 32, 0) == 0      # K not a multiple of 64
-    assert native.w4a16_repack_bytes(4096, 4096, 48, 0) == 0   # group not supported
+    # one record per 128 x 128 unit: 8192 bytes of codes, then G = 128/g groups of 256 bytes of
+    # scales and (asymmetric) 64 bytes of zeros
+    K, N = 4096, 4096
+    units = (K // 128) * (N // 128)
+    for g in (32, 64, 128):
+        G = 128 // g
+        assert native.w4a16_repack_bytes(K, N, g, 0) == units * (8192 + G * 256 + G * 64)
+        assert native.w4a16_repack_bytes(K, N, g, 1) == units * (8192 + G * 256)
+    assert native.w4a16_repack_bytes(K, 8, 128, 0) == 0          # N not a multiple of 128
+    assert native.w4a16_repack_bytes(192, 128, 32, 0) == 0       # K not a multiple of 128
+    assert native.w4a16_repack_bytes(4096, 4096, 48, 0) == 0     # group not supported
 
 
 def test_select_kernel_and_workspace_are_host_only(L):
     for M in (1, 2, 16, 17, 32, 256, 2048):
         k = native.w4a16_select_kernel(M, 4096, 4096, 128)
-        assert k in (native.KERNEL_GEMV, native.KERNEL_TC, native.KERNEL_SKINNY)
-        # decode-sized M streams the weights (GEMV, then the skinny split-K kernel); larger M uses
-        # the tensor-core GEMM
+        assert k in (native.KERNEL_GEMV, native.KERNEL_TC)
+        # decode-sized M streams the weights (the decode GEMV); larger M uses the tensor-core GEMM
         assert k == (native.KERNEL_GEMV if M <= 16 else native.KERNEL_TC)
         assert native.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
     assert native.w4a16_workspace_bytes(0, 4096, 4096, 128) == 0

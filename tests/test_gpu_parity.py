@@ -143,9 +143,11 @@ def test_repack_bit_exact(K, N, group, sym):
     off = oracle.tiled_offsets(K, N, group, sym)
     assert native.w4a16_repack_bytes(K, N, group, sym) == off["total"]
     buf = native.w4a16_repack(gc, gs, gz, K, N, group, sym).cpu().numpy()
-    for region in ("codes", "scales", "zeros"):
-        a, n = off[region], off[region + "_bytes"]
-        assert np.array_equal(buf[a:a + n], ref[a:a + n]), region
+    assert buf.size == ref.size
+    recs, rrec = buf.reshape(-1, off["record"]), ref.reshape(-1, off["record"])
+    for name, a, n in (("codes", 0, off["codes_bytes"]), ("scales", off["scales"], off["scales_bytes"]),
+                       ("zeros", off["zeros"], off["zeros_bytes"])):
+        assert np.array_equal(recs[:, a:a + n], rrec[:, a:a + n]), name
 
 
 # ----------------------------------------------------------------------------- GEMM, small
@@ -334,8 +336,8 @@ def test_gemm_tc_sweep_shape_sampled(M):
 def test_gemm_tc_format_variants_sampled(sym, group, a_dtype):
     K = N = 8192
     Wb, (oc, os_, oz), tiled = _tiled("student_t", K, N, group, sym, 5)
-    for M, kernel in ((16, native.KERNEL_TC), (256, native.KERNEL_TC), (1, native.KERNEL_SKINNY),
-                      (16, native.KERNEL_SKINNY)):
+    for M, kernel in ((16, native.KERNEL_TC), (256, native.KERNEL_TC), (1, native.KERNEL_GEMV),
+                      (4, native.KERNEL_GEMV), (16, native.KERNEL_AUTO)):
         Ab, A = _acts(M, K, 7000 + M, a_dtype)
         cols = synthetic.column_sample(N, 64, seed=M + group + 1)
         C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
@@ -344,9 +346,9 @@ def test_gemm_tc_format_variants_sampled(sym, group, a_dtype):
         _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
 
 
-# ----------------------------------------------------------------------------- tiled layout + skinny tcgen05
-SKINNY_GEMM = [
-    # M, K, N, group, sym, a_dtype    (splits follow from N, K and the group)
+# ----------------------------------------------------------------------------- tiled layout, M <= 16
+DECODE_GEMM = [
+    # M, K, N, group, sym, a_dtype
     (1, 128, 128, 128, 0, 0),         # one unit: no split
     (1, 512, 256, 128, 0, 0),         # the tiny configuration
     (2, 512, 256, 32, 1, 1),
@@ -354,53 +356,8 @@ SKINNY_GEMM = [
     (5, 768, 128, 32, 0, 1),
     (8, 2048, 512, 128, 1, 0),
     (13, 1024, 256, 64, 1, 1),
-    (16, 4096, 1024, 128, 0, 1),
+    (16, 1536, 1024, 128, 0, 1),
 ]
-
-
-@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SKINNY_GEMM)
-def test_gemm_skinny_full_output(M, K, N, group, sym, a_dtype):
-    kind = "student_t" if sym else "normal"
-    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 70 + K + N)
-    Ab, A = _acts(M, K, 800 + M, a_dtype)
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                          kernel=native.KERNEL_SKINNY, dev_status=status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
-
-
-@pytest.mark.parametrize("a_dtype", [0, 1])
-@pytest.mark.parametrize("sym", [0, 1])
-def test_gemm_skinny_unit_rows_return_dequantized_rows(a_dtype, sym):
-    K, N, group = 512, 256, 64
-    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
-    rows = [0, 7, 8, 63, 64, 200, 300, 511, 1, 2, 3, 130, 257, 384, 450, 509]   # 16 rows
-    Ab = np.zeros((len(rows), K), dtype=np.uint16)
-    one = 0x3C00 if a_dtype == 0 else 0x3F80
-    for i, k in enumerate(rows):
-        Ab[i, k] = one
-    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
-    A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                          kernel=native.KERNEL_SKINNY)
-    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
-    expect = oracle.decode16(oracle.encode16(What[rows], a_dtype), a_dtype)   # one rounding
-    got = oracle.decode16(_to_np16(C), a_dtype)
-    assert np.array_equal(got, expect)
-
-
-def test_gemm_skinny_zero_weights_give_zero():
-    K, N, group = 1024, 256, 32
-    W = torch.zeros((K, N), dtype=torch.float16, device="cuda")
-    for sym in (0, 1):
-        gc, gs, gz = native.w4a16_quantize(W, group, sym)
-        tiled = native.w4a16_repack(gc, gs, gz, K, N, group, sym)
-        Ab, A = _acts(7, K, 5, 1)
-        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                              kernel=native.KERNEL_SKINNY)
-        assert torch.count_nonzero(C).item() == 0
 
 
 @pytest.mark.parametrize("K,N", LLAMA8B)
@@ -416,89 +373,9 @@ def test_gemm_llama8b_decode_tiled_sampled(K, N):
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
-def test_gemm_skinny_sweep_shape_sampled(M):
-    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
-    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
-    Ab, A = _acts(M, K, 9000 + M, a_dtype)
-    cols = synthetic.column_sample(N, 96, seed=M + 2)
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                          kernel=native.KERNEL_SKINNY)
-    torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
-
-
-# ----------------------------------------------------------------------------- tiled layout + CUDA-core GEMV
-GEMV_TILED = [
-    # M, K, N, group, sym, a_dtype
-    (1, 512, 256, 128, 0, 0),
-    (1, 384, 128, 128, 1, 1),     # three groups of 64 K tiles
-    (2, 768, 128, 32, 1, 1),
-    (1, 4096, 1024, 64, 0, 1),
-    (2, 2048, 384, 128, 1, 0),
-    (1, 1024, 640, 32, 0, 0),
-    (2, 4096, 256, 64, 0, 1),
-]
-
-
-@pytest.fixture
-def cuda_cores(monkeypatch):
-    monkeypatch.setenv("W4A16_GEMV_VARIANT", "cuda_cores")
-
-
-@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", GEMV_TILED)
-def test_gemm_gemv_tiled_full_output(M, K, N, group, sym, a_dtype, cuda_cores):
-    kind = "student_t" if sym else "normal"
-    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 90 + K + N)
-    Ab, A = _acts(M, K, 1100 + M, a_dtype)
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                          kernel=native.KERNEL_GEMV)
-    torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
-
-
-@pytest.mark.parametrize("a_dtype", [0, 1])
-def test_gemm_gemv_tiled_unit_rows(a_dtype, cuda_cores):
-    K, N, group, sym = 512, 256, 64, 0
-    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
-    What = oracle.dequant(oc, os_, oz, K, N, group, sym)
-    one = 0x3C00 if a_dtype == 0 else 0x3F80
-    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
-    for k in (0, 33, 64, 255, 511):
-        Ab = np.zeros((1, K), dtype=np.uint16)
-        Ab[0, k] = one
-        A = torch.from_numpy(Ab.view(np.int16)).view(tdt).cuda()
-        C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                              kernel=native.KERNEL_GEMV)
-        expect = oracle.decode16(oracle.encode16(What[[k]], a_dtype), a_dtype)
-        assert np.array_equal(oracle.decode16(_to_np16(C), a_dtype), expect)
-
-
-@pytest.mark.parametrize("M", [1, 2])
-def test_gemm_gemv_sweep_shape_sampled(M, cuda_cores):
-    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
-    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
-    Ab, A = _acts(M, K, 9500 + M, a_dtype)
-    cols = synthetic.column_sample(N, 128, seed=M + 3)
-    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
-                          kernel=native.KERNEL_GEMV)
-    torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
-
-
-@pytest.fixture(params=["stream", "cluster"])
-def mma_variant(request, monkeypatch):
-    if request.param == "cluster":
-        monkeypatch.setenv("W4A16_GEMV_VARIANT", "cluster")
-    else:
-        monkeypatch.delenv("W4A16_GEMV_VARIANT", raising=False)
-    return request.param
-
-
-@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", SKINNY_GEMM)
-def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype, mma_variant):
-    """The decode kernels (warp-level MMA: persistent stream-K and cluster split-K) at M = 1..16
-    on the tiled layout."""
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", DECODE_GEMM)
+def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype):
+    """The decode kernel (persistent stream-K, warp-level MMA) at M = 1..16 on the tiled layout."""
     kind = "student_t" if sym else "normal"
     Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 70 + K + N)
     Ab, A = _acts(M, K, 1300 + M, a_dtype)
@@ -508,8 +385,8 @@ def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype, mma_variant):
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
-@pytest.mark.parametrize("M", [4, 9, 16])
-def test_gemm_gemv_mma_sweep_shape_sampled(M, mma_variant):
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_gemm_gemv_mma_sweep_shape_sampled(M):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9700 + M, a_dtype)
@@ -525,12 +402,12 @@ STREAM_GEMM = [
     # M, K, N, group, sym, a_dtype      (units = N/128 * K/128 against one CTA per SM)
     (1, 128, 128, 128, 0, 0),           # one unit, one CTA
     (1, 8192, 128, 128, 0, 1),          # one tile cut among 64 CTAs
-    (3, 16384, 256, 128, 1, 0),         # two tiles, each cut among about 74 CTAs
+    (2, 16384, 256, 128, 1, 0),         # two tiles, each cut among about 74 CTAs
     (1, 4096, 1024, 32, 0, 0),          # 256 units: tiles cut in two
     (8, 2048, 1280, 64, 1, 1),
     (9, 1024, 2560, 128, 0, 1),         # two n8 tiles of rows
-    (16, 3072, 768, 32, 1, 0),
-    (1, 14336, 512, 128, 1, 1),         # long K, symmetric reference chains
+    (16, 1024, 768, 32, 1, 0),
+    (1, 14336, 512, 128, 1, 1),         # long K, symmetric
     (2, 4096, 6144, 128, 0, 0),         # every CTA holds whole tiles and cut ones
 ]
 
@@ -560,7 +437,7 @@ def test_gemm_stream_full_output(M, K, N, group, sym, a_dtype):
 @pytest.mark.parametrize("group", [128, 32])
 def test_gemm_stream_unit_rows_return_dequantized_rows(a_dtype, sym, group):
     """A = unit rows: each output row is one dequantized weight row rounded once, bit for bit,
-    also through the reference-chain correction of group 128."""
+    through the post-scaled (group 128) and the pre-scaled (group 32) paths."""
     K, N = 1024, 384
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 41)
     rows = [0, 1, 2, 3, 8, 9, 31, 32, 63, 64, 127, 128, 500, 777, 1022, 1023]
@@ -580,8 +457,8 @@ def test_gemm_stream_unit_rows_return_dequantized_rows(a_dtype, sym, group):
 
 @pytest.mark.parametrize("a_dtype", [0, 1])
 def test_gemm_stream_zero_weights_give_exact_zero(a_dtype):
-    """All-zero weight columns give exactly zero (the bound there is 1e-5 absolute), for the
-    asymmetric (code 0, zero 0) and symmetric (offset-binary 8) references."""
+    """All-zero weight columns give exactly zero (the bound there is 1e-5 absolute), asymmetric
+    (code 0, zero 0) and symmetric (offset-binary code 8, zero 8): u - z is exactly 0."""
     K, N = 2048, 512
     W = torch.zeros((K, N), dtype=torch.float16, device="cuda")
     W[:, 256:] = torch.from_numpy(synthetic.weights_normal(K, 256, seed=3).view(np.int16)).view(
@@ -605,6 +482,19 @@ def test_gemm_stream_llama70b_decode_sampled(K, N):
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 3000 + N)
     Ab, A = _acts(1, K, 4000 + K, a_dtype)
     cols = synthetic.column_sample(N, 256, seed=K + N + 7)
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
+    torch.cuda.synchronize()
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("M", [6, 8, 9, 16])
+def test_gemm_auto_sweep_shape_sampled_skinny(M):
+    """M rows of A too long for the decode kernel's shared memory: the AUTO dispatch takes the
+    tensor-core GEMM, still within the bound."""
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 9900 + M, a_dtype)
+    cols = synthetic.column_sample(N, 96, seed=M + 5)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)

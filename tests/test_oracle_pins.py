@@ -404,59 +404,64 @@ def _slots(word):
 
 
 def test_tiled_layout_positions_and_bijection(oracle_mod):
-    """The tiled buffer is a permutation of the plain words: each word lands once, at the
-    position the layout's definition gives (closed forms for chosen words), with its codes in
-    slot order (e0, e2, e4, e6, e1, e3, e5, e7)."""
+    """The tiled buffer is a permutation of the plain words into unit records: each word lands
+    once, at the byte the layout's definition gives (closed forms for chosen words: unit record
+    t * K/128 + c, block h at 2048 h, channel slot n XOR 2h, word w), with its codes in slot
+    order (e0, e2, e4, e6, e1, e3, e5, e7); every record carries its unit's scales and zeros."""
     K, N, group = 256, 384, 64
+    G = 128 // group
     rows = K // 8
-    nwords = rows * N
-    # every plain word carries its own index in bits 8..31 and the element number in the
-    # low byte pattern 0x10 (element 0 = 0, element 1 = 1): make element e's nibble = e
     rng = np.random.default_rng(17)
     codes = rng.integers(-2**31, 2**31, size=(rows, N), dtype=np.int64).astype(np.int32)
     scales = np.arange((K // group) * N, dtype=np.uint16).reshape(K // group, N)
     zeros = np.arange((K // group) * (N // 8), dtype=np.int32).reshape(K // group, N // 8)
     buf = oracle_mod.repack(codes, scales, zeros, K, N, group, False)
     off = oracle_mod.tiled_offsets(K, N, group, False)
-    words = buf[: off["codes_bytes"]].view(np.int32)
-    assert words.size == nwords
-    ktiles = K // 64
+    R = off["record"]
+    assert R == 8192 + G * 256 + G * 64 and off["total"] == (N // 128) * (K // 128) * R
+    assert off["zeros_bytes"] == G * 64 and oracle_mod.tiled_offsets(K, N, group, True)["zeros_bytes"] == 0
+    assert oracle_mod.tiled_offsets(K, N, group, True)["record"] == 8192 + G * 256
+    assert len(buf) == off["total"]
 
-    def plain_elems(j, n):
-        return _slots(np.uint32(codes[j, n]))
+    def word_at(byte):
+        return int(buf[byte: byte + 4].view(np.uint32)[0])
 
-    def check(pos, j, n):
-        e = plain_elems(j, n)
-        assert _slots(np.uint32(words[pos])) == [e[0], e[2], e[4], e[6], e[1], e[3], e[5], e[7]]
+    def check(byte, j, n):
+        e = _slots(np.uint32(codes[j, n]))
+        assert _slots(word_at(byte)) == [e[0], e[2], e[4], e[6], e[1], e[3], e[5], e[7]]
 
-    check(0, 0, 0)
-    check(1, 1, 0)           # four consecutive rows of one channel in 16 bytes
-    check(3, 3, 0)
-    check(4, 0, 1)           # then the next channel
-    check(512, 4, 0)         # second half of the tile: rows 4..7
-    check(1024, 8, 0)        # next tile along K
-    check(ktiles * 1024, 0, 128)   # next 128 channels
-    check(ktiles * 1024 + 1024 + 512 + 4 * 5 + 2, 8 + 4 + 2, 128 + 5)
-    # a bijection: decode every tiled word back and compare the multiset of plain words
-    def decode(t):
-        s_ = _slots(np.uint32(t))
+    check(0, 0, 0)                      # record 0, block 0, channel 0, word 0
+    check(4, 1, 0)                      # four consecutive rows of one channel in 16 bytes
+    check(12, 3, 0)
+    check(16, 0, 1)                     # then the next channel (slot 1 XOR 0)
+    check(2048 + 16 * 2, 4, 0)          # block 1 (rows 4..7): channel 0 sits in slot 0 XOR 2
+    check(2048 + 16 * 0, 4, 2)          # ... and channel 2 in slot 2 XOR 2 = 0
+    check(3 * 2048 + 16 * (5 ^ 6) + 8, 12 + 2, 5)      # block 3, slot 5 XOR 6, word 2
+    check(R, 16, 0)                     # next record along K
+    check(2 * R + 16 * 1, 0, 129)                      # t = 1, c = 0: record 1 * K/128 + 0
+    check(3 * R + 2048 + 16 * (1 ^ 2) + 4, 21, 129)   # t = 1, c = 1, block 1, word 1
+    # a bijection: decode every code word of every record and compare the multisets
+    def decode(tw):
+        s_ = _slots(np.uint32(tw))
         e = [s_[0], s_[4], s_[1], s_[5], s_[2], s_[6], s_[3], s_[7]]
         return sum(v << (4 * i) for i, v in enumerate(e))
-    back = np.array(sorted(decode(t) for t in words), dtype=np.int64)
+    recs = buf.reshape(-1, R)
+    words = recs[:, :8192].copy().view(np.uint32).reshape(-1)
+    back = np.array(sorted(decode(tw) for tw in words), dtype=np.int64)
     assert np.array_equal(back, np.sort((codes.astype(np.int64) & 0xFFFFFFFF).reshape(-1)))
-    assert off["scales"] % 256 == 0 and off["zeros"] % 256 == 0 and off["total"] % 256 == 0
-    assert off["scales"] >= off["codes_bytes"]
-    assert np.array_equal(buf[off["scales"]: off["scales"] + off["scales_bytes"]].view(np.uint16),
-                          scales.reshape(-1))
-    assert np.array_equal(buf[off["zeros"]: off["zeros"] + off["zeros_bytes"]].view(np.int32),
-                          zeros.reshape(-1))
-    offs = oracle_mod.tiled_offsets(K, N, group, True)
-    assert offs["zeros_bytes"] == 0
+    # scales and zeros of unit (t, c): plain group rows c*G .. c*G + G-1, the tile's channels
+    for t in range(N // 128):
+        for c in range(K // 128):
+            rec = recs[t * (K // 128) + c]
+            sc = rec[8192: 8192 + G * 256].copy().view(np.uint16).reshape(G, 128)
+            zr = rec[8192 + G * 256:].copy().view(np.int32).reshape(G, 16)
+            assert np.array_equal(sc, scales[c * G: c * G + G, 128 * t: 128 * t + 128])
+            assert np.array_equal(zr, zeros[c * G: c * G + G, 16 * t: 16 * t + 16])
 
 
 def test_tiled_layout_symmetric_is_offset_binary(oracle_mod):
     """Symmetric codes -8..7 are stored as q + 8 (0..15) in the tiled buffer."""
-    K, N, group = 64, 128, 32
+    K, N, group = 128, 128, 32
     q = np.tile(np.arange(-8, 8), 4 * N // 16 * K // 4)[: K * N].reshape(K, N)
     words = np.zeros((K // 8, N), dtype=np.int64)
     for k in range(K):

@@ -8,7 +8,6 @@ from .native import (  # noqa: F401
     F16,
     KERNEL_AUTO,
     KERNEL_GEMV,
-    KERNEL_SKINNY,
     KERNEL_TC,
     LAYOUT_PLAIN,
     LAYOUT_TILED,

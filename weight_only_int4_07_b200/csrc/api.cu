@@ -32,7 +32,6 @@ int forced_kernel() {
         const char* e = getenv("W4A16_FORCE_KERNEL");
         if (e && strcmp(e, "gemv") == 0) forced = W4A16_KERNEL_GEMV;
         if (e && strcmp(e, "tc") == 0) forced = W4A16_KERNEL_TC;
-        if (e && strcmp(e, "skinny") == 0) forced = W4A16_KERNEL_SKINNY;
     });
     return forced;
 }
@@ -51,17 +50,17 @@ const char* kernel_name(int k) {
     switch (k) {
         case W4A16_KERNEL_GEMV: return "gemv";
         case W4A16_KERNEL_TC: return "tc";
-        case W4A16_KERNEL_SKINNY: return "skinny";
         default: return "auto";
     }
 }
 
 // The dispatch proper (tiled layout), without the environment override. Up to M = 16 the layer is
-// bound by the weight stream and the split-K skinny kernel serves it; above, the tensor-core GEMM.
+// bound by the weight stream and the stream-K decode GEMV serves it; above, the tensor-core GEMM.
 int dispatch(int M, int N, int K, int group) {
     (void)N;
+    (void)K;
     (void)group;
-    return (M <= 16 && K % 128 == 0) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_TC;
+    return M <= 16 ? W4A16_KERNEL_GEMV : W4A16_KERNEL_TC;
 }
 
 }  // namespace
@@ -100,7 +99,7 @@ W4A16_API int w4a16_quantize(const void* W, int K, int N, int group, int sym, in
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym) {
     if (check_shape(K, N, group) != W4A16_OK || (sym != 0 && sym != 1)) return 0;
     if (N % kTileN != 0 || K % kTileK != 0) return 0;
-    return tiled_offsets(K, N, group, sym).total;
+    return tiled_layout(K, N, group, sym).total;
 }
 
 W4A16_API int w4a16_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K,
@@ -130,7 +129,7 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group) {
     const GemvPlan p = plan_gemv_plain(M, N, K, group);
     int n_sm = gemv_stream_sm_count();
     if (n_sm <= 0) n_sm = 148;
-    const GemvStreamPlan q = plan_gemv_stream(M, N, K, group, n_sm);
+    const GemvStreamPlan q = plan_gemv_stream(M, N, K, group, 0, n_sm);   // asymmetric: the larger plan
     const size_t rest = q.ok && q.partial_bytes > p.ws_bytes ? q.partial_bytes : p.ws_bytes;
     return kGemvStreamCounterBytes + rest;
 }
@@ -145,8 +144,7 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
     if (a_dtype != W4A16_F16 && a_dtype != W4A16_BF16) return W4A16_EINVAL;
     if (layout != W4A16_LAYOUT_PLAIN && layout != W4A16_LAYOUT_TILED) return W4A16_EINVAL;
     if (sym != 0 && sym != 1) return W4A16_EINVAL;
-    if (kernel != W4A16_KERNEL_AUTO && kernel != W4A16_KERNEL_GEMV && kernel != W4A16_KERNEL_TC &&
-        kernel != W4A16_KERNEL_SKINNY)
+    if (kernel != W4A16_KERNEL_AUTO && kernel != W4A16_KERNEL_GEMV && kernel != W4A16_KERNEL_TC)
         return W4A16_EINVAL;
     if (!A || !wq || !C) return W4A16_EINVAL;
     if (layout == W4A16_LAYOUT_PLAIN) {
@@ -184,26 +182,14 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
         return W4A16_OK;
     }
     if (chosen == W4A16_KERNEL_GEMV && layout == W4A16_LAYOUT_TILED) {
-        const char* variant = getenv("W4A16_GEMV_VARIANT");
-        if (variant && strcmp(variant, "cuda_cores") == 0) {
-            st = launch_gemv_tiled(A, a_dtype, M, K, wq, N, group, sym, C, s);
-        } else if (variant && strcmp(variant, "cluster") == 0) {
-            st = launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
-        } else {
-            st = launch_gemv_stream(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
-            // activations of M rows too long for shared memory: the cluster split-K kernel
-            if (st == W4A16_EUNSUPPORTED) st = launch_gemv_mma(A, a_dtype, M, K, wq, N, group, sym, C, s);
-        }
-        // M > 16, or activations too long for one split's shared memory: the tensor-core kernel
+        st = launch_gemv_stream(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
+        // M > 16, or M rows of A too long for shared memory: the tensor-core kernel
         if (st == W4A16_EUNSUPPORTED && kernel == W4A16_KERNEL_AUTO)
             return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
         return st;
     }
     if (chosen == W4A16_KERNEL_TC && layout == W4A16_LAYOUT_TILED) {
         return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
-    }
-    if (chosen == W4A16_KERNEL_SKINNY && layout == W4A16_LAYOUT_TILED && M <= 16) {
-        return launch_gemm_skinny(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
     }
     return W4A16_EUNSUPPORTED;
 }

@@ -65,15 +65,6 @@ int launch_gemv_plain(const void* A, int a_dtype, int M, int K, const int32_t* c
 int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                    void* C, int* dev_status, cudaStream_t stream);
 
-int launch_gemm_skinny(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
-                       void* C, int* dev_status, cudaStream_t stream);
-
-int launch_gemv_tiled(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
-                      void* C, cudaStream_t stream);
-
-int launch_gemv_mma(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
-                    void* C, cudaStream_t stream);
-
 // Persistent stream-K decode kernel. Its workspace starts with one int counter per 128-channel
 // tile (kGemvStreamCounterBytes, zero between calls; each call leaves them zero), followed by
 // the FP32 partial sums of tiles cut between CTAs.
@@ -83,10 +74,10 @@ struct GemvStreamPlan {
     bool ok;
     int ns;               // pipeline stages
     int ctas;             // persistent CTAs (one per SM)
-    size_t act_bytes, ref_bytes, red_bytes, smem;
+    size_t row_bytes, act_bytes, red_bytes, stage_bytes, smem;
     size_t partial_bytes; // workspace after the counters
 };
-GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int n_sm);
+GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm);
 int gemv_stream_sm_count();
 int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                        void* C, void* workspace, int* dev_status, cudaStream_t stream);

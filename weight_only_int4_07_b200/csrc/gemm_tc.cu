@@ -13,8 +13,9 @@
 //
 // Warp roles (192 threads):
 //   warp 0      : one thread issues, per 64-K stage, a TMA tile load of the activations
-//                 (128-byte swizzle), a bulk copy of the stage's 4 KiB code tile from the tiled
-//                 weight buffer, and bulk copies of the stage's scales and zeros.
+//                 (128-byte swizzle), a bulk copy of the stage's 4 KiB of codes (half of a unit
+//                 record of the tiled buffer), and bulk copies of the stage's scales and zeros
+//                 from the same record.
 //   warp 1      : allocates tensor memory; one thread issues the four tcgen05.mma of a stage
 //                 and commits them to the stage's "empty" barrier.
 //   warps 2..5  : dequantize -- one thread per output channel turns its 64 codes of the stage
@@ -103,8 +104,7 @@ struct Deq<__nv_bfloat16> {
 template <int BN, typename T>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restrict__ tiled, int M, int K,
-               int N, int group, int sym, uint32_t scales_off, uint32_t zeros_off, T* __restrict__ C,
-               int* dev_status) {
+               int N, int group, int sym, const TiledLayout L, T* __restrict__ C, int* dev_status) {
     using Cfg = TcCfg<BN>;
     constexpr int NS = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -156,15 +156,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
                 uint8_t* st = smem + s * Cfg::kStage;
                 mbar_arrive_expect_tx(&full[s], stage_bytes);
                 tma_2d_g2s(st + Cfg::kA, &tmA, it * 64, m0, &full[s]);
-                bulk_g2s(st + Cfg::kA + Cfg::kB, tiled + ((size_t)nt * kstages + it) * 4096, 4096, &full[s]);
-                const int g0 = (it * 64) / group;
-                for (int j = 0; j < groups_per_stage; ++j) {
-                    bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes + j * 256,
-                             tiled + scales_off + ((size_t)(g0 + j) * N + n0) * 2, 256, &full[s]);
-                    if (!sym)
-                        bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales + j * 64,
-                                 tiled + zeros_off + ((size_t)(g0 + j) * (N / 8) + n0 / 8) * 4, 64, &full[s]);
-                }
+                // unit record (nt, it / 2): blocks 2 (it % 2), 2 (it % 2) + 1 of its codes, and
+                // the record's groups that fall in this stage (contiguous in the record)
+                const uint8_t* rec = tiled + ((size_t)nt * (K / 128) + it / 2) * L.record;
+                bulk_g2s(st + Cfg::kA + Cfg::kB, rec + (it & 1) * 4096, 4096, &full[s]);
+                const int lg0 = (it * 64) / group - (it / 2) * L.groups;
+                bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes, rec + L.scales + lg0 * 256, groups_per_stage * 256,
+                         &full[s]);
+                if (!sym)
+                    bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales, rec + L.zeros + lg0 * 64,
+                             groups_per_stage * 64, &full[s]);
                 ++issued;
             }
             // drain: every copy issued has landed before the block may exit
@@ -214,7 +215,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restric
             const __half* ssm = reinterpret_cast<const __half*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes);
             const uint32_t* zsm = reinterpret_cast<const uint32_t*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales);
             uint8_t* atile = st;
-            const uint4 w4 = ctile[128 * hf + n];   // rows 4 hf .. 4 hf + 3 of the stage
+            // rows 4 hf .. 4 hf + 3 of the stage: block h = 2 (it % 2) + hf of the unit record,
+            // channel n in slot n ^ 2h
+            const uint4 w4 = ctile[128 * hf + (n ^ (2 * (2 * (it & 1) + hf)))];
             const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
             // group of this half inside the stage (group 32: one group per half)
             const int lg = groups_per_stage > 1 ? hf : 0;
@@ -313,11 +316,10 @@ int launch_tc_typed(const void* A, int M, int K, const void* tiled, int N, int g
     if (attr_err != cudaSuccess) return W4A16_ECUDA;
     CUtensorMap map;
     if (!make_act_map(&map, A, M, K, BN, !std::is_same<T, __half>::value)) return W4A16_ECUDA;
-    const TiledOffsets off = tiled_offsets(K, N, group, sym);
+    const TiledLayout L = tiled_layout(K, N, group, sym);
     dim3 grid(N / 128, (M + BN - 1) / BN);
     tc_gemm_kernel<BN, T><<<grid, kThreadsTC, Cfg::kSmem, stream>>>(
-        map, static_cast<const uint8_t*>(tiled), M, K, N, group, sym, (uint32_t)off.scales,
-        (uint32_t)off.zeros, static_cast<T*>(C), dev_status);
+        map, static_cast<const uint8_t*>(tiled), M, K, N, group, sym, L, static_cast<T*>(C), dev_status);
     return launch_status();
 }
 

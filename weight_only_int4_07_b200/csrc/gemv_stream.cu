@@ -5,37 +5,32 @@
 // weight byte crosses HBM once, with data movement overlapped with compute); "INT8 vs INT4
 // Quantization, in depth", "Two regimes" (at small batch the layer waits for memory).
 //
-// Work split. The weights are a sequence of units, one unit = one 128-channel tile x one 128-K
-// step (8 KiB of codes), ordered tile-major. One CTA per SM takes a contiguous range of
-// floor(U / P) or ceil(U / P) units, so every SM streams the same number of bytes whatever the
-// shape. A tile whose units all belong to one CTA is written straight to C; a tile cut between
-// CTAs is finished by the last of them to arrive (a counter per tile in the workspace), which
-// adds the FP32 partial sums of all of them in CTA order, so the result does not depend on timing.
+// Work split. The weights are the tiled buffer's unit records (128 channels x 128 K, codes then
+// scales then zeros), ordered tile-major, so a contiguous range of units is one contiguous range
+// of bytes. One CTA per SM takes floor(U / P) or ceil(U / P) consecutive units. A tile whose units
+// all belong to one CTA is written straight to C; a tile cut between CTAs is finished by the last
+// of them to arrive (a counter per tile in the workspace), which adds the FP32 partial sums of
+// all of them in CTA order, so the result does not depend on timing.
 //
-// Bytes in flight. Warp 16 (one thread) keeps `ns` (8..16) stages of bulk copies in flight: per
-// unit the four 2 KiB half-tiles of codes (to shared-memory offsets 2048 + 32 bytes apart, which
-// makes the consumers' 16-byte reads bank-conflict free) and the unit's scales and zero-points.
-// Sixteen consumer warps in two groups take the units alternately (group = unit parity).
+// Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each;
+// the last warp to leave a stage refills it with the stage ns positions later, so no warp waits
+// for another to issue a copy. Sixteen warps in four groups: group q takes unit q of every stage,
+// warp w of a group owns channels 32 w .. 32 w + 31 of the unit.
 //
-// Math (warp-level tensor-core MMA, m16n8k16, FP32 accumulators). Warp w of a group owns channels
-// 16 w .. 16 w + 15 of the tile; lane (g = lane / 4, t = lane % 4) reads the 32 K of half-tile t
-// for channels 16 w + g and 16 w + g + 8 and batch rows 8 b + g of A. Nibble pairs become 16-bit
-// operands by one mask-OR with a magic exponent: fp16 0x6400 | u = 1024 + u, and for the nibble
-// one position up 0x6400 | (u << 4) = 1024 + 16 u; bf16 0x4300 | u = 128 + u (its 7-bit mantissa
-// has no room for the shifted form). Two MMA chains per unit: chain A takes the 1024 + u operands,
-// chain B the 1024 + 16 u ones (bf16: both chains 128 + u).
-// Group size 128 (one group per unit): the chains run on the raw operands. The same chains with
-// every code at its zero reference (u = 0; offset-binary 8 for symmetric codes) give R_A and R_B;
-// these depend only on A, are computed once per CTA and unit into shared memory, and
-//   sum_k a_k (u_k - z) = (acc_A - R_A f_A) + (acc_B - R_B f_B) / 16,
-// f_A = (1024 + z) / (1024 + z_ref), f_B = (1024 + 16 z) / (1024 + 16 z_ref), both exact in FP32.
-// A group whose codes all equal the reference has acc = R bit for bit (the same MMAs on the same
-// operands), so an all-zero group contributes exactly zero. The FP32 sum is scaled by s[g, n].
-// Smaller groups (several per unit): each operand is dequantized before the MMA, (u - z) exact in
-// the 16-bit type, then times s rounded once (bf16: s = s_hi + s_lo, both exact in bf16).
-//
-// Every mbarrier wait is bounded (2 s); on expiry the kernel records W4A16_ETIMEOUT and skips
-// its remaining work, still passing every CTA barrier and tile counter.
+// Math (warp-level tensor-core MMA, m16n8k16, FP32 accumulators), per warp and unit: lane
+// (g = lane / 4, t = lane % 4) reads the 16 bytes of block t (32 K) of channels 32 w + g + 8 r,
+// r = 0..3 (block t keeps channel n at slot n ^ 2t: the four lanes t of a channel hit different
+// banks), and the unit's activations of batch rows 8 b + g. Nibble pairs become 16-bit operands
+// by one mask-OR with a magic exponent: fp16 0x6400 | u = 1024 + u, and for the nibble one
+// position up 0x6400 | (u << 4) = 1024 + 16 u (no shift); bf16 0x4300 | u = 128 + u. The zero
+// point is subtracted exactly in 16 bits: (1024 + u) - (1024 + z), (1024 + 16 u) / 16 - (64 + z),
+// (128 + u) - (128 + z). Group 128: the MMAs accumulate sum a (u - z) of the unit in FP32, and
+// the unit's scale multiplies that sum once. Groups 64 and 32 (a lane's 32 K may span several
+// groups): each operand is scaled first, (u - z) * s rounded once to the 16-bit type (bf16:
+// s = s_hi + s_lo, both exact in bf16), and the MMAs accumulate the whole tile segment.
+// Every mbarrier wait is bounded (2 s); on expiry the kernel records W4A16_ETIMEOUT, stops
+// issuing copies, still passes every CTA barrier and tile counter, and lets the copies in
+// flight land before it exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -47,56 +42,57 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kGsGroupWarps = 8;                         // warps per consumer group (128 channels)
-constexpr int kGsConsumers = 2 * kGsGroupWarps;          // two groups: even and odd units
-constexpr int kGsThreads = 32 * (kGsConsumers + 1);      // + one producer warp
-constexpr int kGsHalf = 2048 + 32;                       // skewed half-tile stride in a stage
-constexpr int kGsScalesOff = 4 * kGsHalf;                // up to 4 groups x 256 B
-constexpr int kGsZerosOff = kGsScalesOff + 4 * 256;      // up to 4 groups x 64 B
-constexpr int kGsStage = kGsZerosOff + 4 * 64;           // 9600 bytes
-constexpr int kGsMinStages = 6, kGsMaxStages = 16;
+constexpr int kGsGroups = 4, kGsGroupWarps = 4, kGsWarps = kGsGroups * kGsGroupWarps;
+constexpr int kGsThreads = 32 * kGsWarps;
+constexpr int kGsUnitsPerStage = kGsGroups;
+constexpr int kGsMinStages = 3, kGsMaxStages = 16;
 constexpr int kGsSmemMax = 227 * 1024;
 constexpr uint64_t kGsSpin = 2000000000ull;
 
-static_assert(kGsStage % 128 == 0, "stage size");
+__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {   // a >> k for b = 2^(32-k)
+    uint32_t r;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
 
-// 16-bit operand handling per activation type.
+__device__ __forceinline__ uint32_t andor(uint32_t a, uint32_t b, uint32_t c) {   // (a & b) | c
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// Masks and shift multipliers, passed at run time so that the compiler keeps them in registers:
+// one lop3 per operand register, shifts on the multiply pipe.
+struct GsMasks {
+    uint32_t lo, hi, magic, m4, m8, m12;
+};
+
 template <typename T>
 struct GsOps;
 
 template <>
 struct GsOps<__half> {
-    static constexpr uint32_t kMagic = 0x64006400u;
-    static constexpr float kInvB = 1.0f / 16.0f;           // chain B carries 16 u
-    static __device__ __forceinline__ uint32_t ref_a(int zr) { return (uint32_t)(0x6400 + zr) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t ref_b(int zr) { return (uint32_t)(0x6400 + 16 * zr) * 0x00010001u; }
-    static __device__ __forceinline__ float fa(int z) { return fmaf((float)z, 1.0f / 1024.0f, 1.0f); }
-    static __device__ __forceinline__ float fb(int z) { return fmaf((float)z, 1.0f / 64.0f, 1.0f); }
-    // nibble pairs of one word: r0 (elements 0,1) and r2 (4,5) for chain A, r1 (2,3) and r3 (6,7) for B
-    static __device__ __forceinline__ void unpack(uint32_t w, uint32_t (&r)[4]) {
-        const uint32_t h = w >> 8;
-        r[0] = (w & 0x000F000Fu) | kMagic;
-        r[1] = (w & 0x00F000F0u) | kMagic;
-        r[2] = (h & 0x000F000Fu) | kMagic;
-        r[3] = (h & 0x00F000F0u) | kMagic;
+    // operands: r0 = elements (0,1), r2 = (4,5) as 1024 + u; r1 = (2,3), r3 = (6,7) as 1024 + 16 u
+    static __device__ __forceinline__ void unpack(uint32_t w, const GsMasks& k, uint32_t (&r)[4]) {
+        const uint32_t h = mulhi(w, k.m8);
+        r[0] = andor(w, k.lo, k.magic);
+        r[1] = andor(w, k.hi, k.magic);
+        r[2] = andor(h, k.lo, k.magic);
+        r[3] = andor(h, k.hi, k.magic);
     }
-    // exact (u - z) for chain A / chain B operands
-    static __device__ __forceinline__ uint32_t zz_a(int z) { return (uint32_t)(0x6400 + z) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t zz_b(int z) {  // -(64 + z), packed
-        __half2 h = __floats2half2_rn(-(64.0f + (float)z), -(64.0f + (float)z));
-        return *reinterpret_cast<uint32_t*>(&h);
-    }
-    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {
+    static __device__ __forceinline__ uint32_t zz_a(uint32_t z) { return (0x6400u + z) * 0x00010001u; }
+    static __device__ __forceinline__ uint32_t zz_b(uint32_t z) { return (0xD400u + (z << 4)) * 0x00010001u; }
+    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {   // (1024+u) - (1024+z)
         uint32_t r;
         asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(zz));
         return r;
     }
-    static __device__ __forceinline__ uint32_t sub_b(uint32_t x, uint32_t zz) {  // x / 16 - (64 + z)
+    static __device__ __forceinline__ uint32_t sub_b(uint32_t x, uint32_t zz) {   // x / 16 - (64 + z)
         uint32_t r;
         asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(0x2C002C00u), "r"(zz));
         return r;
     }
-    struct Scale {
+    struct Scale {   // d * s, one rounding (s is an fp16 value)
         uint32_t s2;
         __device__ __forceinline__ void set(uint16_t bits) { s2 = (uint32_t)bits * 0x00010001u; }
         __device__ __forceinline__ uint32_t apply(uint32_t d) const {
@@ -116,27 +112,22 @@ struct GsOps<__half> {
 
 template <>
 struct GsOps<__nv_bfloat16> {
-    static constexpr uint32_t kMagic = 0x43004300u;
-    static constexpr float kInvB = 1.0f;
-    static __device__ __forceinline__ uint32_t ref_a(int zr) { return (uint32_t)(0x4300 + zr) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t ref_b(int zr) { return ref_a(zr); }
-    static __device__ __forceinline__ float fa(int z) { return fmaf((float)z, 1.0f / 128.0f, 1.0f); }
-    static __device__ __forceinline__ float fb(int z) { return fa(z); }
-    static __device__ __forceinline__ void unpack(uint32_t w, uint32_t (&r)[4]) {
-        r[0] = (w & 0x000F000Fu) | kMagic;
-        r[1] = ((w >> 4) & 0x000F000Fu) | kMagic;
-        r[2] = ((w >> 8) & 0x000F000Fu) | kMagic;
-        r[3] = ((w >> 12) & 0x000F000Fu) | kMagic;
+    // operands: all four registers as 128 + u (elements (0,1), (2,3), (4,5), (6,7))
+    static __device__ __forceinline__ void unpack(uint32_t w, const GsMasks& k, uint32_t (&r)[4]) {
+        r[0] = andor(w, k.lo, k.magic);
+        r[1] = andor(mulhi(w, k.m4), k.lo, k.magic);
+        r[2] = andor(mulhi(w, k.m8), k.lo, k.magic);
+        r[3] = andor(mulhi(w, k.m12), k.lo, k.magic);
     }
-    static __device__ __forceinline__ uint32_t zz_a(int z) { return (uint32_t)(0x4300 + z) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t zz_b(int z) { return zz_a(z); }
-    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {
+    static __device__ __forceinline__ uint32_t zz_a(uint32_t z) { return (0x4300u + z) * 0x00010001u; }
+    static __device__ __forceinline__ uint32_t zz_b(uint32_t z) { return zz_a(z); }
+    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {   // (128+u) - (128+z)
         uint32_t r;
         asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(zz));
         return r;
     }
     static __device__ __forceinline__ uint32_t sub_b(uint32_t x, uint32_t zz) { return sub_a(x, zz); }
-    struct Scale {  // d * s rounded once: s = s_hi (bf16 truncation of s) + s_lo (exact in bf16)
+    struct Scale {   // d * s rounded once: s = s_hi (bf16 truncation of s) + s_lo (exact in bf16)
         uint32_t hi2, lo2;
         __device__ __forceinline__ void set(uint16_t bits) {
             const float s = __half2float(__ushort_as_half(bits));
@@ -164,24 +155,17 @@ struct GsOps<__nv_bfloat16> {
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
-
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
-// First unit of CTA c when U units are cut into P contiguous ranges.
+// First unit of CTA c when U units are cut into P contiguous ranges, and the CTA holding unit u.
 __device__ __forceinline__ long long unit_begin(int c, long long U, int P) { return ((long long)c * U) / P; }
-// The CTA whose range holds unit u.
-__device__ __forceinline__ int unit_owner(long long u, long long U, int P) {
-    return (int)(((u + 1) * P - 1) / U);
-}
+__device__ __forceinline__ int unit_owner(long long u, long long U, int P) { return (int)(((u + 1) * P - 1) / U); }
 
-// Byte offset of A[m, k] (k a multiple of 8) in the shared activation copy: rows of 2K + 32 bytes,
-// each 128-K unit 256 bytes, and inside it the 16-byte chunk q of 32-K block t stored at
-// position (q + t / 2) mod 4 (conflict-free 16-byte reads by the MMA lanes).
-__device__ __forceinline__ uint32_t act_offset(int m, int k, uint32_t row_bytes) {
-    const int kk = k & 127, t = kk >> 5, q = (kk >> 3) & 3;
-    return (uint32_t)m * row_bytes + (uint32_t)(k >> 7) * 256u + (uint32_t)t * 64u +
-           (uint32_t)((q + (t >> 1)) & 3) * 16u;
+// Warp-uniform bounded wait: the common case (phase already complete) costs one try and a vote.
+__device__ __forceinline__ bool wait_uniform(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, kGsSpin));
 }
 
 struct GsParams {
@@ -191,366 +175,319 @@ struct GsParams {
     int* counters;      // one int per tile, zero between calls
     float* partials;    // [P][2][M][128]
     int* dev_status;
-    unsigned long long scales_off, zeros_off;
     int M, K, N, sym, ns, P;
-    uint32_t row_bytes;   // 2 K + 32
-    uint32_t act_bytes, ref_bytes, red_bytes;
+    uint32_t record, scales_off, zeros_off;
+    uint32_t stage_bytes, row_bytes, act_bytes, red_bytes;
+    GsMasks km;
 };
 
-template <int NB, typename T, int GROUP>
+// NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
+template <int NB, typename T, int GROUP, bool ODD>
 __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     using Ops = GsOps<T>;
-    constexpr int MT = 8 * NB;
-    constexpr bool kRef = (GROUP == 128);
-    constexpr int G = GROUP >= 128 ? 1 : 128 / GROUP;   // groups per unit
+    constexpr bool kPost = (GROUP == 128);   // one group per unit: scale the unit's sum
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int M = p.M, K = p.K, N = p.N, ns = p.ns, P = p.P;
     const int steps = K / 128;
-    const int tiles = N / 128;
-    const long long U = (long long)tiles * steps;
+    const long long U = (long long)(N / 128) * steps;
     const int cta = blockIdx.x;
     const long long u0 = unit_begin(cta, U, P), u1 = unit_begin(cta + 1, U, P);
+    const int nunits = (int)(u1 - u0);
+    const uint32_t R = p.record, stage_bytes = p.stage_bytes, RS = p.row_bytes;
 
-    uint8_t* acts = smem_raw;                                               // [M][2K + 32] rotated
-    float* refs = reinterpret_cast<float*>(smem_raw + p.act_bytes);         // [steps][2][MT]
-    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes + p.ref_bytes);       // [MT][128]
-    uint8_t* stages = smem_raw + p.act_bytes + p.ref_bytes + p.red_bytes;  // ns x kGsStage
-    uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * kGsStage);
+    uint8_t* acts = smem_raw;                                             // [M][RS]
+    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][3][M][128]
+    uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes;                 // 320 zero bytes
+    uint8_t* stages = zrow + 384;                                         // ns x stage_bytes
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);
     uint64_t* empty = full + ns;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + ns);
-    volatile int* last_flag = abort_flag + 1;
+    int* flags = reinterpret_cast<int*>(empty + ns);
+    volatile int* abort_flag = flags;
+    volatile int* last_flag = flags + 1;
+    int* issued = flags + 2;            // [ns] copies issued into each slot
+    int* leave = flags + 2 + ns;        // [ns] warps that have left the slot's current stage
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kGsGroupWarps);
+            mbar_init(&empty[i], kGsThreads);
+            issued[i] = 0;
+            leave[i] = 0;
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
+    for (int i = threadIdx.x; i < 96; i += kGsThreads) reinterpret_cast<uint32_t*>(zrow)[i] = 0u;
     __syncthreads();
     grid_dependents_launch();
 
-    if (warp == kGsConsumers) {
-        // ------------------------------------------------------------------------ producer
-        if (lane == 0) {
-            const int ktiles = K / 64;
-            const uint32_t bytes = 8192u + (uint32_t)G * (256u + (p.sym ? 0u : 64u));
-            int s = 0;
-            uint32_t ph = 0;
-            long long issued = 0;
-            int tile = (int)(u0 / steps), sp = (int)(u0 - (long long)tile * steps);
-            for (long long u = u0; u < u1; ++u) {
-                if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.dev_status, kGsSpin)) break;
-                uint8_t* st = stages + (size_t)s * kGsStage;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                const uint8_t* src = p.tiled + ((size_t)tile * ktiles + 2 * (size_t)sp) * 4096;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) bulk_g2s(st + b * kGsHalf, src + b * 2048, 2048, &full[s]);
-#pragma unroll
-                for (int gg = 0; gg < G; ++gg) {
-                    const size_t gi = (size_t)sp * G + gg;
-                    bulk_g2s(st + kGsScalesOff + 256 * gg, p.tiled + p.scales_off + (gi * N + (size_t)tile * 128) * 2,
-                             256, &full[s]);
-                    if (!p.sym)
-                        bulk_g2s(st + kGsZerosOff + 64 * gg,
-                                 p.tiled + p.zeros_off + (gi * (N / 8) + (size_t)tile * 16) * 4, 64, &full[s]);
-                }
-                ++issued;
-                if (++s == ns) { s = 0; ph ^= 1u; }
-                if (++sp == steps) { sp = 0; ++tile; }
-            }
-            // copies still in flight land before the CTA exits (only a cut-short run has any)
-            const long long first = issued > ns ? issued - ns : 0;
-            for (long long i = first; i < issued; ++i)
-                mbar_wait(&full[i % ns], (uint32_t)((i / ns) & 1), abort_flag, p.dev_status, kGsSpin);
-        }
-        return;
-    }
+    // stage st = records u0 + 4 st .. (up to 4), one bulk copy into slot st % ns
+    const int nst = (nunits + kGsUnitsPerStage - 1) / kGsUnitsPerStage;
+    auto issue = [&](int st) {
+        const int s = st % ns;
+        const int n = nunits - st * kGsUnitsPerStage < kGsUnitsPerStage ? nunits - st * kGsUnitsPerStage
+                                                                        : kGsUnitsPerStage;
+        const uint32_t bytes = (uint32_t)n * R;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_g2s(stages + (size_t)s * stage_bytes, p.tiled + (size_t)(u0 + (long long)st * kGsUnitsPerStage) * R,
+                 bytes, &full[s]);
+        atomicAdd(&issued[s], 1);
+    };
+    if (threadIdx.x == 0)
+        for (int st = 0; st < nst && st < ns; ++st) issue(st);
 
-    // ---------------------------------------------------------------------------- consumers
-    const int grp = warp / kGsGroupWarps;           // 0: even units, 1: odd units
-    const int wg = warp % kGsGroupWarps;            // channel block of the warp
-    const int ctid = threadIdx.x;                   // 0 .. 511
+    const int grp = warp / kGsGroupWarps, wg = warp % kGsGroupWarps;
     const int g = lane >> 2, t = lane & 3;
-    const int ch0 = 16 * wg + g, ch1 = ch0 + 8;
-    const int zr = p.sym ? 8 : 0;
+    const int ch0 = 32 * wg + g;     // this lane's channels: ch0 + 8 r, r = 0..3
     const T* A = static_cast<const T*>(p.A);
 
     // A may be the output of the previous kernel in the stream
     grid_dependency_wait();
     {
+        // activations: 32-K block t of unit sp at sp * 320 + 80 t (the 16-byte padding makes the
+        // lanes' 16-byte reads conflict free); pairs in each 16-byte chunk stored (p0, p2, p1, p3)
+        // so that each MMA's two B registers are adjacent; each CTA starts at a different chunk
         const int vpr = K / 8;
         for (int m = 0; m < M; ++m)
-            for (int c = ctid; c < vpr; c += 32 * kGsConsumers)
-                *reinterpret_cast<uint4*>(acts + act_offset(m, 8 * c, p.row_bytes)) =
-                    *reinterpret_cast<const uint4*>(A + (size_t)m * K + 8 * c);
-    }
-    named_bar(1, 32 * kGsConsumers);
-
-    // activation fragments of one unit: lane holds row 8 b + g, K 32 t .. 32 t + 31 of the unit
-    auto load_b = [&](int sp, uint32_t (&bfr)[NB][16]) {
+            for (int c0 = threadIdx.x; c0 < vpr; c0 += 4 * kGsThreads) {
+                uint4 vv[4];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int row = 8 * b + g;
-            if (row < M) {
-                const uint8_t* base = acts + (uint32_t)row * p.row_bytes + (uint32_t)sp * 256u + (uint32_t)t * 64u;
+                for (int j = 0; j < 4; ++j)
+                    if (c0 + j * kGsThreads < vpr)
+                        vv[j] = *reinterpret_cast<const uint4*>(A + (size_t)m * K +
+                                                                 8 * ((c0 + j * kGsThreads + cta * 64) % vpr));
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(base + ((q + (t >> 1)) & 3) * 16);
-                    bfr[b][4 * q + 0] = v.x;
-                    bfr[b][4 * q + 1] = v.y;
-                    bfr[b][4 * q + 2] = v.z;
-                    bfr[b][4 * q + 3] = v.w;
-                }
-            } else {
-#pragma unroll
-                for (int r = 0; r < 16; ++r) bfr[b][r] = 0u;
+                for (int j = 0; j < 4; ++j)
+                    if (c0 + j * kGsThreads < vpr) {
+                        const int c = (c0 + j * kGsThreads + cta * 64) % vpr;
+                        const uint32_t off = (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u +
+                                             (uint32_t)((c >> 2) & 3) * 80u + (uint32_t)(c & 3) * 16u;
+                        *reinterpret_cast<uint4*>(acts + off) = make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
+                    }
             }
-        }
+    }
+    __syncthreads();
+
+    // activation fragments: lane holds row 8 b + g (rows at or past M read a zero block)
+    const uint8_t* abase[NB];
+    uint32_t astride[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const bool real = 8 * b + g < M;
+        abase[b] = real ? acts + (uint32_t)(8 * b + g) * RS + (uint32_t)t * 80u : zrow + (uint32_t)t * 80u;
+        astride[b] = real ? 320u : 0u;
+    }
+
+    const GsMasks km = p.km;
+    const int lg = kPost ? 0 : (32 * t) / GROUP;                                  // group of block t
+    const uint32_t coff = (uint32_t)t * 2048u + (uint32_t)(ch0 ^ (2 * t)) * 16u;   // channel ch0 + 8 r: + 128 r
+    const uint32_t soff = p.scales_off + 256u * (uint32_t)lg + 2u * (uint32_t)ch0; // + 16 r
+    const uint32_t zoff = p.zeros_off + 64u * (uint32_t)lg + 16u * (uint32_t)wg;   // words of ch0 + 8 r
+    const int zsh = 4 * g;
+    const uint32_t rec_off = (uint32_t)grp * R;
+    const int sym = p.sym;
+
+    float tot[2][NB][4];
+    auto zero_tot = [&]() {
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) tot[rt][b][0] = tot[rt][b][1] = tot[rt][b][2] = tot[rt][b][3] = 0.0f;
     };
+    zero_tot();
+    int tile = (int)(u0 / steps);
+    int seg_lo = 0, sp_lo = (int)(u0 - (long long)tile * steps);
+    int seg_hi = (steps - sp_lo) < nunits ? (steps - sp_lo) : nunits;
 
-    if constexpr (kRef) {
-        // R_A, R_B of every unit this CTA touches: the chains below with all codes at the reference
-        const long long span = u1 - u0;
-        const int nref = span >= steps ? steps : (int)span;
-        const int sp_first = (int)(u0 % steps);
-        const uint32_t ca = Ops::ref_a(zr), cb = Ops::ref_b(zr);
-        for (int i = warp; i < nref; i += kGsConsumers) {
-            int sp = sp_first + i;
-            if (sp >= steps) sp -= steps;
-            uint32_t bfr[NB][16];
-            load_b(sp, bfr);
+    // end of a tile segment: groups 1..3 hand their sums to group 0 through shared memory (two
+    // buffers, by tile parity, so one CTA barrier per tile suffices); group 0 writes C, or this
+    // CTA's partial sums when the tile is cut between CTAs
+    auto emit = [&]() {
+        float* rb = red + (size_t)(tile & 1) * 3 * M * 128;
+        if (grp > 0) {
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    Ops::mma(ra, ca, ca, ca, ca, bfr[b][4 * j + 0], bfr[b][4 * j + 2]);
-                    Ops::mma(rb, cb, cb, cb, cb, bfr[b][4 * j + 1], bfr[b][4 * j + 3]);
-                }
-                if (g == 0) {  // row 0 of the MMA; columns 2t, 2t + 1 = batch rows 8 b + 2t (+1)
-                    float* r = refs + (size_t)sp * 2 * MT;
-                    r[8 * b + 2 * t] = ra[0];
-                    r[8 * b + 2 * t + 1] = ra[1];
-                    r[MT + 8 * b + 2 * t] = rb[0];
-                    r[MT + 8 * b + 2 * t + 1] = rb[1];
-                }
-            }
-        }
-        named_bar(1, 32 * kGsConsumers);
-    }
-
-    const int lgi = GROUP >= 128 ? 0 : (32 * t) / GROUP;   // group of this lane's 32 K inside a unit
-    const int zsh0 = 4 * (ch0 & 7), zsh1 = 4 * (ch1 & 7);
-    bool aborted = false;
-    int s = grp;                 // stage of this group's next unit (ns is even)
-    uint32_t ph = 0;
-    long long u = u0;
-    while (u < u1) {
-        const int tile = (int)(u / steps);
-        const long long seg_end = ((long long)tile + 1) * steps < u1 ? ((long long)tile + 1) * steps : u1;
-        float tot[NB][4], tot2[NB][4];
+                for (int b = 0; b < NB; ++b)
 #pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) tot[b][e] = tot2[b][e] = 0.0f;
-
-        for (long long uu = u + (((u - u0) & 1) != grp ? 1 : 0); uu < seg_end; uu += 2) {
-            if (!aborted && !mbar_wait(&full[s], ph, abort_flag, p.dev_status, kGsSpin)) aborted = true;
-            if (!aborted) {
-                const int sp = (int)(uu - (long long)tile * steps);
-                const uint8_t* st = stages + (size_t)s * kGsStage;
-                const uint4 w0 = *reinterpret_cast<const uint4*>(st + t * kGsHalf + ch0 * 16);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(st + t * kGsHalf + ch1 * 16);
-                const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + kGsScalesOff + 256 * lgi);
-                const uint16_t sb0 = sc[ch0], sb1 = sc[ch1];
-                int z0 = zr, z1 = zr;
-                if (!p.sym) {
-                    const uint32_t* zw = reinterpret_cast<const uint32_t*>(st + kGsZerosOff + 64 * lgi);
-                    z0 = (int)((zw[ch0 >> 3] >> zsh0) & 0xFu);
-                    z1 = (int)((zw[ch1 >> 3] >> zsh1) & 0xFu);
-                }
-                uint32_t bfr[NB][16];
-                load_b(sp, bfr);
-                float2 ra[NB], rb[NB];
-                if constexpr (kRef) {
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const float* r = refs + (size_t)sp * 2 * MT;
-                        ra[b] = *reinterpret_cast<const float2*>(r + 8 * b + 2 * t);
-                        rb[b] = *reinterpret_cast<const float2*>(r + MT + 8 * b + 2 * t);
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                        if (m < M) rb[((grp - 1) * M + m) * 128 + ch] = tot[rt][b][e];
                     }
-                }
-                // the stage is in registers: let the producer refill it
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-
-                const uint32_t wr0[4] = {w0.x, w0.y, w0.z, w0.w};
-                const uint32_t wr1[4] = {w1.x, w1.y, w1.z, w1.w};
-                if constexpr (kRef) {
-                    float acc_a[NB][4], acc_b[NB][4];
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc_a[b][e] = acc_b[b][e] = 0.0f;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t q0[4], q1[4];
-                        Ops::unpack(wr0[j], q0);
-                        Ops::unpack(wr1[j], q1);
-#pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            Ops::mma(acc_a[b], q0[0], q1[0], q0[2], q1[2], bfr[b][4 * j + 0], bfr[b][4 * j + 2]);
-                            Ops::mma(acc_b[b], q0[1], q1[1], q0[3], q1[3], bfr[b][4 * j + 1], bfr[b][4 * j + 3]);
-                        }
-                    }
-                    const float s0 = __half2float(__ushort_as_half(sb0));
-                    const float s1 = __half2float(__ushort_as_half(sb1));
-                    const float fa0 = p.sym ? 1.0f : Ops::fa(z0), fa1 = p.sym ? 1.0f : Ops::fa(z1);
-                    const float fb0 = p.sym ? 1.0f : Ops::fb(z0), fb1 = p.sym ? 1.0f : Ops::fb(z1);
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        // elements: 0, 1 -> channel ch0, batch rows 2t, 2t+1; 2, 3 -> channel ch1
-                        const float d0 = fmaf(fmaf(-rb[b].x, fb0, acc_b[b][0]), Ops::kInvB, fmaf(-ra[b].x, fa0, acc_a[b][0]));
-                        const float d1 = fmaf(fmaf(-rb[b].y, fb0, acc_b[b][1]), Ops::kInvB, fmaf(-ra[b].y, fa0, acc_a[b][1]));
-                        const float d2 = fmaf(fmaf(-rb[b].x, fb1, acc_b[b][2]), Ops::kInvB, fmaf(-ra[b].x, fa1, acc_a[b][2]));
-                        const float d3 = fmaf(fmaf(-rb[b].y, fb1, acc_b[b][3]), Ops::kInvB, fmaf(-ra[b].y, fa1, acc_a[b][3]));
-                        tot[b][0] = fmaf(s0, d0, tot[b][0]);
-                        tot[b][1] = fmaf(s0, d1, tot[b][1]);
-                        tot[b][2] = fmaf(s1, d2, tot[b][2]);
-                        tot[b][3] = fmaf(s1, d3, tot[b][3]);
-                    }
-                } else {
-                    const uint32_t za0 = Ops::zz_a(z0), za1 = Ops::zz_a(z1);
-                    const uint32_t zb0 = Ops::zz_b(z0), zb1 = Ops::zz_b(z1);
-                    typename Ops::Scale sc0, sc1;
-                    sc0.set(sb0);
-                    sc1.set(sb1);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t q0[4], q1[4];
-                        Ops::unpack(wr0[j], q0);
-                        Ops::unpack(wr1[j], q1);
-                        q0[0] = sc0.apply(Ops::sub_a(q0[0], za0));
-                        q0[2] = sc0.apply(Ops::sub_a(q0[2], za0));
-                        q0[1] = sc0.apply(Ops::sub_b(q0[1], zb0));
-                        q0[3] = sc0.apply(Ops::sub_b(q0[3], zb0));
-                        q1[0] = sc1.apply(Ops::sub_a(q1[0], za1));
-                        q1[2] = sc1.apply(Ops::sub_a(q1[2], za1));
-                        q1[1] = sc1.apply(Ops::sub_b(q1[1], zb1));
-                        q1[3] = sc1.apply(Ops::sub_b(q1[3], zb1));
-#pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            Ops::mma(tot[b], q0[0], q1[0], q0[2], q1[2], bfr[b][4 * j + 0], bfr[b][4 * j + 2]);
-                            Ops::mma(tot2[b], q0[1], q1[1], q0[3], q1[3], bfr[b][4 * j + 1], bfr[b][4 * j + 3]);
-                        }
-                    }
-                }
-            }
-            s += 2;
-            if (s >= ns) { s -= ns; ph ^= 1u; }
         }
-
-        // ---------------------------------------------------------------- segment output
-        if constexpr (!kRef) {
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) tot[b][e] += tot2[b][e];
-        }
-        // group 1 hands its sums to group 0 through shared memory
-        if (grp == 1) {
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int m = 8 * b + 2 * t;
-                red[m * 128 + ch0] = tot[b][0];
-                red[(m + 1) * 128 + ch0] = tot[b][1];
-                red[m * 128 + ch1] = tot[b][2];
-                red[(m + 1) * 128 + ch1] = tot[b][3];
-            }
-        }
-        named_bar(1, 32 * kGsConsumers);
-        if (grp == 0) {
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int m = 8 * b + 2 * t;
-                tot[b][0] += red[m * 128 + ch0];
-                tot[b][1] += red[(m + 1) * 128 + ch0];
-                tot[b][2] += red[m * 128 + ch1];
-                tot[b][3] += red[(m + 1) * 128 + ch1];
-            }
-        }
-        named_bar(1, 32 * kGsConsumers);
+        __syncthreads();
         if (grp == 0) {
             T* C = static_cast<T*>(p.C);
             const size_t n0 = (size_t)tile * 128;
-            const int c_first = unit_owner((long long)tile * steps, U, P);
-            const int c_last = unit_owner((long long)tile * steps + steps - 1, U, P);
-            if (c_first == c_last) {
+            const int cf = unit_owner((long long)tile * steps, U, P);
+            const int cl = unit_owner((long long)tile * steps + steps - 1, U, P);
+            float* part = p.partials + ((size_t)cta * 2 + (tile == (int)(u0 / steps) ? 0 : 1)) * (size_t)M * 128;
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    const int m = 8 * b + 2 * t;
-                    if (m < M) {
-                        C[(size_t)m * N + n0 + ch0] = Act<T>::from_f32(tot[b][0]);
-                        C[(size_t)m * N + n0 + ch1] = Act<T>::from_f32(tot[b][2]);
-                    }
-                    if (m + 1 < M) {
-                        C[(size_t)(m + 1) * N + n0 + ch0] = Act<T>::from_f32(tot[b][1]);
-                        C[(size_t)(m + 1) * N + n0 + ch1] = Act<T>::from_f32(tot[b][3]);
-                    }
-                }
-            } else {
-                // partial sums of this CTA for the tile: slot 0 if it is the CTA's first tile
-                const int slot = (tile == (int)(u0 / steps)) ? 0 : 1;
-                float* part = p.partials + ((size_t)cta * 2 + slot) * (size_t)M * 128;
+            for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    const int m = 8 * b + 2 * t;
-                    if (m < M) {
-                        part[(size_t)m * 128 + ch0] = tot[b][0];
-                        part[(size_t)m * 128 + ch1] = tot[b][2];
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                        if (m < M) {
+                            const float v = tot[rt][b][e] + rb[m * 128 + ch] + rb[(M + m) * 128 + ch] +
+                                            rb[(2 * M + m) * 128 + ch];
+                            if (cf == cl) C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(v);
+                            else part[m * 128 + ch] = v;
+                        }
                     }
-                    if (m + 1 < M) {
-                        part[(size_t)(m + 1) * 128 + ch0] = tot[b][1];
-                        part[(size_t)(m + 1) * 128 + ch1] = tot[b][3];
-                    }
-                }
-                __threadfence();
+            if (cf != cl) {
+                // the last CTA of the tile to arrive adds every CTA's partial sums in CTA order
                 named_bar(2, 32 * kGsGroupWarps);
-                if (ctid == 0) {
-                    const int old = atomicAdd(&p.counters[tile], 1);
-                    *last_flag = (old == c_last - c_first) ? 1 : 0;
+                if (threadIdx.x == 0) {
+                    int old;
+                    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + tile)
+                                 : "memory");
+                    *last_flag = (old == cl - cf) ? 1 : 0;
                 }
                 named_bar(2, 32 * kGsGroupWarps);
                 if (*last_flag) {
-                    // the last CTA of the tile adds every CTA's partial sums in CTA order
-                    __threadfence();
-                    for (int e = ctid; e < M * 128; e += 32 * kGsGroupWarps) {
+                    for (int e = threadIdx.x; e < M * 128; e += 32 * kGsGroupWarps) {
                         float sum = 0.0f;
-                        for (int c = c_first; c <= c_last; ++c) {
+                        for (int c = cf; c <= cl; ++c) {
                             const int sl = (tile == (int)(unit_begin(c, U, P) / steps)) ? 0 : 1;
                             sum += __ldcg(p.partials + ((size_t)c * 2 + sl) * (size_t)M * 128 + e);
                         }
                         C[(size_t)(e >> 7) * N + n0 + (e & 127)] = Act<T>::from_f32(sum);
                     }
-                    if (ctid == 0) p.counters[tile] = 0;
+                    if (threadIdx.x == 0) p.counters[tile] = 0;
                 }
-                named_bar(2, 32 * kGsGroupWarps);
             }
         }
-        u = seg_end;
+        zero_tot();
+        ++tile;
+        sp_lo = 0;
+        seg_lo = seg_hi;
+        seg_hi = seg_lo + steps < nunits ? seg_lo + steps : nunits;
+    };
+
+    bool aborted = false;
+    int s_idx = -1;
+    uint32_t ph = 0;
+    for (int st = 0; st < nst; ++st) {
+        if (st > 0 && !aborted) {
+            // leave stage st - 1; the last warp to leave refills the slot with stage st - 1 + ns
+            mbar_arrive(&empty[s_idx]);
+            __syncwarp();
+            bool bad = false;
+            if (lane == 0 && atomicAdd(&leave[s_idx], 1) == kGsWarps - 1) {
+                leave[s_idx] = 0;
+                const int r = st - 1;
+                if (r + ns < nst) {
+                    if (mbar_wait(&empty[s_idx], (uint32_t)(r / ns) & 1u, abort_flag, p.dev_status, kGsSpin)) issue(r + ns);
+                    else bad = true;
+                }
+            }
+            if (__any_sync(0xffffffffu, bad)) aborted = true;
+        }
+        if (++s_idx == ns) {
+            s_idx = 0;
+            ph ^= 1u;
+        }
+        if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status)) aborted = true;
+        const int li = st * kGsUnitsPerStage + grp;
+        if (li >= nunits) continue;
+        while (li >= seg_hi) emit();
+        if (aborted) continue;
+        const int sp = sp_lo + (li - seg_lo);
+        const uint8_t* rec = stages + (uint32_t)s_idx * stage_bytes + rec_off;
+        uint4 cw[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cw[r] = *reinterpret_cast<const uint4*>(rec + coff + 128 * r);
+        uint16_t sb[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sb[r] = *reinterpret_cast<const uint16_t*>(rec + soff + 16 * r);
+        uint4 zw = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);   // symmetric: z = 8
+        if (!sym) zw = *reinterpret_cast<const uint4*>(rec + zoff);
+        uint4 v[NB][4];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const uint8_t* a = abase[b] + (uint32_t)sp * astride[b];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[b][i] = *reinterpret_cast<const uint4*>(a + 16 * i);
+        }
+        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
+            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
+            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+            const uint32_t z0 = (zws[2 * rt] >> zsh) & 0xFu, z1 = (zws[2 * rt + 1] >> zsh) & 0xFu;
+            const uint32_t za0 = Ops::zz_a(z0), za1 = Ops::zz_a(z1), zb0 = Ops::zz_b(z0), zb1 = Ops::zz_b(z1);
+            typename Ops::Scale sc0, sc1;
+            if constexpr (!kPost) {
+                sc0.set(sb[2 * rt]);
+                sc1.set(sb[2 * rt + 1]);
+            }
+            float acc[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t q0[4], q1[4];
+                Ops::unpack(w0[i], km, q0);
+                Ops::unpack(w1[i], km, q1);
+                q0[0] = Ops::sub_a(q0[0], za0);
+                q0[2] = Ops::sub_a(q0[2], za0);
+                q0[1] = Ops::sub_b(q0[1], zb0);
+                q0[3] = Ops::sub_b(q0[3], zb0);
+                q1[0] = Ops::sub_a(q1[0], za1);
+                q1[2] = Ops::sub_a(q1[2], za1);
+                q1[1] = Ops::sub_b(q1[1], zb1);
+                q1[3] = Ops::sub_b(q1[3], zb1);
+                if constexpr (!kPost) {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        q0[x] = sc0.apply(q0[x]);
+                        q1[x] = sc1.apply(q1[x]);
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    float (&d)[4] = kPost ? acc[b] : tot[rt][b];
+                    Ops::mma(d, q0[0], q1[0], q0[2], q1[2], v[b][i].x, v[b][i].y);
+                    Ops::mma(d, q0[1], q1[1], q0[3], q1[3], v[b][i].z, v[b][i].w);
+                }
+            }
+            if constexpr (kPost) {
+                const float s0 = __half2float(__ushort_as_half(sb[2 * rt]));
+                const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1]));
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    tot[rt][b][0] = fmaf(s0, acc[b][0], tot[rt][b][0]);
+                    tot[rt][b][2] = fmaf(s1, acc[b][2], tot[rt][b][2]);
+                    if (ODD) {
+                        tot[rt][b][1] = fmaf(s0, acc[b][1], tot[rt][b][1]);
+                        tot[rt][b][3] = fmaf(s1, acc[b][3], tot[rt][b][3]);
+                    }
+                }
+            }
+        }
+    }
+    while (seg_lo < nunits) emit();
+
+    // after a timeout: let every copy still in flight land before the CTA exits (a wait that
+    // does not give up on the raised abort flag, still bounded in time)
+    if (threadIdx.x == 0 && *abort_flag) {
+        volatile int keep_waiting = 0;
+        for (int s = 0; s < ns; ++s)
+            if (issued[s] > 0) mbar_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u, &keep_waiting, nullptr, kGsSpin);
     }
 }
 
-template <int NB, typename T, int GROUP>
+template <int NB, typename T, int GROUP, bool ODD>
 int launch_typed(const GsParams& prm, size_t smem, cudaStream_t stream) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<NB, T, GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kGsSmemMax);
+        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<NB, T, GROUP, ODD>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kGsSmemMax);
     });
     if (attr_err != cudaSuccess) return W4A16_ECUDA;
     cudaLaunchConfig_t cfg = {};
@@ -563,25 +500,31 @@ int launch_typed(const GsParams& prm, size_t smem, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_stream_kernel<NB, T, GROUP>, prm);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_stream_kernel<NB, T, GROUP, ODD>, prm);
     return e == cudaSuccess ? W4A16_OK : W4A16_ECUDA;
 }
 
-template <int NB, typename T>
+template <int NB, typename T, bool ODD>
 int launch_group(const GsParams& prm, int group, size_t smem, cudaStream_t stream) {
     switch (group) {
-        case 32: return launch_typed<NB, T, 32>(prm, smem, stream);
-        case 64: return launch_typed<NB, T, 64>(prm, smem, stream);
-        case 128: return launch_typed<NB, T, 128>(prm, smem, stream);
+        case 32: return launch_typed<NB, T, 32, ODD>(prm, smem, stream);
+        case 64: return launch_typed<NB, T, 64, ODD>(prm, smem, stream);
+        case 128: return launch_typed<NB, T, 128, ODD>(prm, smem, stream);
         default: return W4A16_EUNSUPPORTED;
     }
+}
+
+template <typename T>
+int launch_rows(const GsParams& prm, int group, size_t smem, cudaStream_t stream) {
+    if (prm.M > 8) return launch_group<2, T, true>(prm, group, smem, stream);
+    if (prm.M > 1) return launch_group<1, T, true>(prm, group, smem, stream);
+    return launch_group<1, T, false>(prm, group, smem, stream);
 }
 
 int sm_count() {
     static int cached[64] = {0};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev < 0 || dev >= 64) return 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (cached[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
@@ -592,26 +535,27 @@ int sm_count() {
 
 }  // namespace
 
-GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int n_sm) {
+GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm) {
     GemvStreamPlan pl = {};
     if (M < 1 || M > 16 || K % 128 != 0 || N % 128 != 0 || K < 128 || N < 128) return pl;
     if (group != 32 && group != 64 && group != 128) return pl;
     if (N / 128 > kGemvStreamMaxTiles) return pl;
-    const int nb = M <= 8 ? 1 : 2;
-    const size_t row_bytes = 2 * (size_t)K + 32;
-    pl.act_bytes = ((size_t)M * row_bytes + 127) & ~(size_t)127;
-    pl.ref_bytes = group == 128 ? (((size_t)(K / 128) * 2 * 8 * nb * 4 + 127) & ~(size_t)127) : 0;
-    pl.red_bytes = (size_t)8 * nb * 128 * 4;
-    const size_t fixed = pl.act_bytes + pl.ref_bytes + pl.red_bytes + 2 * kGsMaxStages * 8 + 16;
+    const TiledLayout L = tiled_layout(K, N, group, sym);
+    const size_t units = (size_t)(K / 128);
+    pl.row_bytes = 320 * units + ((units & 1) ? 0 : 64);          // 80-byte blocks; rows 64 mod 128 apart
+    pl.act_bytes = ((size_t)M * pl.row_bytes + 127) & ~(size_t)127;
+    pl.red_bytes = (size_t)2 * 3 * M * 128 * 4;
+    pl.stage_bytes = ((size_t)kGsUnitsPerStage * L.record + 127) & ~(size_t)127;
+    const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 8 + 8 * kGsMaxStages + 127) & ~(size_t)127;
+    const size_t fixed = pl.act_bytes + pl.red_bytes + 384 + flags;
     if (fixed >= (size_t)kGsSmemMax) return pl;
-    size_t ns = ((size_t)kGsSmemMax - fixed) / (kGsStage + 16);
+    size_t ns = ((size_t)kGsSmemMax - fixed) / pl.stage_bytes;
     if (ns > kGsMaxStages) ns = kGsMaxStages;
-    ns &= ~(size_t)1;
     if (ns < kGsMinStages) return pl;
     pl.ns = (int)ns;
-    pl.smem = pl.act_bytes + pl.ref_bytes + pl.red_bytes + ns * kGsStage + 2 * ns * 8 + 16;
-    const long long units = (long long)(N / 128) * (K / 128);
-    pl.ctas = n_sm > 0 ? (int)(units < n_sm ? units : n_sm) : 0;
+    pl.smem = fixed + ns * pl.stage_bytes;
+    const long long total_units = (long long)(N / 128) * (K / 128);
+    pl.ctas = n_sm > 0 ? (int)(total_units < n_sm ? total_units : n_sm) : 0;
     pl.partial_bytes = (size_t)(n_sm > 0 ? n_sm : 0) * 2 * M * 128 * 4;
     pl.ok = pl.ctas > 0;
     return pl;
@@ -621,10 +565,10 @@ int gemv_stream_sm_count() { return sm_count(); }
 
 int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                        void* C, void* workspace, int* dev_status, cudaStream_t stream) {
-    const GemvStreamPlan pl = plan_gemv_stream(M, N, K, group, sm_count());
+    const GemvStreamPlan pl = plan_gemv_stream(M, N, K, group, sym, sm_count());
     if (!pl.ok) return W4A16_EUNSUPPORTED;
     if (!workspace) return W4A16_EWORKSPACE;
-    const TiledOffsets off = tiled_offsets(K, N, group, sym);
+    const TiledLayout L = tiled_layout(K, N, group, sym);
     GsParams prm = {};
     prm.A = A;
     prm.tiled = static_cast<const uint8_t*>(tiled);
@@ -632,24 +576,28 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.counters = static_cast<int*>(workspace);
     prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kGemvStreamCounterBytes);
     prm.dev_status = dev_status;
-    prm.scales_off = off.scales;
-    prm.zeros_off = off.zeros;
     prm.M = M;
     prm.K = K;
     prm.N = N;
     prm.sym = sym;
     prm.ns = pl.ns;
     prm.P = pl.ctas;
-    prm.row_bytes = (uint32_t)(2 * (size_t)K + 32);
+    prm.record = L.record;
+    prm.scales_off = L.scales;
+    prm.zeros_off = L.zeros;
+    prm.stage_bytes = (uint32_t)pl.stage_bytes;
+    prm.row_bytes = (uint32_t)pl.row_bytes;
     prm.act_bytes = (uint32_t)pl.act_bytes;
-    prm.ref_bytes = (uint32_t)pl.ref_bytes;
     prm.red_bytes = (uint32_t)pl.red_bytes;
-    if (a_dtype == W4A16_BF16) {
-        if (M <= 8) return launch_group<1, __nv_bfloat16>(prm, group, pl.smem, stream);
-        return launch_group<2, __nv_bfloat16>(prm, group, pl.smem, stream);
-    }
-    if (M <= 8) return launch_group<1, __half>(prm, group, pl.smem, stream);
-    return launch_group<2, __half>(prm, group, pl.smem, stream);
+    const bool bf16 = a_dtype == W4A16_BF16;
+    prm.km.lo = 0x000F000Fu;
+    prm.km.hi = bf16 ? 0x000F000Fu : 0x00F000F0u;
+    prm.km.magic = bf16 ? 0x43004300u : 0x64006400u;
+    prm.km.m4 = 1u << 28;
+    prm.km.m8 = 1u << 24;
+    prm.km.m12 = 1u << 20;
+    if (bf16) return launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream);
+    return launch_rows<__half>(prm, group, pl.smem, stream);
 }
 
 }  // namespace w4a16

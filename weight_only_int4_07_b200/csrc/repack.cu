@@ -1,20 +1,10 @@
-// repack.cu -- one-time permutation of the plain packed codes into the tiled layout.
+// repack.cu -- one-time permutation of the plain packed weight into the tiled layout of unit
+// records (tiled_layout.cuh).
 //
 // "INT4 and Low-Bit Inference", section 5 "The kernel is half the story": weights are permuted
 // once at load so that unpacking is branch-free and coalesced. "4.3 Weight-only INT4", section 4:
-// weights pre-reordered into a layout that suits runtime reads.
-//
-// Tile (t, c): output channels [128 t, 128 t + 128), packed rows j in [8 c, 8 c + 8)
-// (input channels [64 c, 64 c + 64)); tile index t * (K / 64) + c; 1024 words per tile.
-// Word (j, n) of the plain layout goes to word offset, inside its tile,
-//     ((j % 8) / 4) * 512 + (n % 128) * 4 + (j % 4)
-// so a 16-byte vector holds four consecutive packed rows of one output channel and 32
-// consecutive channels read 512 contiguous bytes. Inside each word the eight codes are
-// re-ordered (tiled_encode_word): nibble slot p holds element 2p and slot p + 4 holds element
-// 2p + 1 (p = 0..3), so that one mask of the word yields two adjacent K elements in the two
-// 16-bit halves of a register. Symmetric codes are stored offset-binary (q + 8, zero-point 8).
-// Scales and zeros are copied unchanged after the codes, each region starting on a 256-byte
-// boundary. Nothing is rounded: a bijection of bits.
+// weights pre-reordered into a layout that suits runtime reads. Nothing is rounded: a bijection
+// of the code bits, plus copies of the scales and zeros into the records of their units.
 #include "common.cuh"
 #include "tiled_layout.cuh"
 
@@ -22,35 +12,49 @@ namespace w4a16 {
 
 namespace {
 
-__global__ void repack_codes_kernel(const int32_t* __restrict__ codes, int K, int N, int sym,
-                                    int32_t* __restrict__ tiled) {
-    // one thread per plain word, in plain order: coalesced reads, 16-byte-grouped writes
+__global__ void repack_codes_kernel(const int32_t* __restrict__ codes, int K, int N, int sym, uint32_t record,
+                                    uint8_t* __restrict__ tiled) {
+    // one thread per plain word, in plain order: coalesced reads
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t total = (size_t)(K / 8) * N;
     if (idx >= total) return;
     const int j = (int)(idx / N);
     const int n = (int)(idx - (size_t)j * N);
-    tiled[tiled_word_offset(j, n, K)] = (int32_t)tiled_encode_word((uint32_t)codes[idx], sym);
+    *reinterpret_cast<uint32_t*>(tiled + tiled_word_byte(j, n, K, record)) =
+        tiled_encode_word((uint32_t)codes[idx], sym);
+}
+
+// One thread per (group row, channel): the scale, and for the first channel of each 8 the zeros
+// word, into the record of the unit that holds the group.
+__global__ void repack_meta_kernel(const uint16_t* __restrict__ scales, const int32_t* __restrict__ zeros, int K,
+                                   int N, int group, TiledLayout L, uint8_t* __restrict__ tiled) {
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t total = (size_t)(K / group) * N;
+    if (idx >= total) return;
+    const int gi = (int)(idx / N);
+    const int n = (int)(idx - (size_t)gi * N);
+    const int c = gi / L.groups, gg = gi % L.groups;
+    const int t = n / kTileN, nl = n % kTileN;
+    uint8_t* rec = tiled + ((size_t)t * (K / kTileK) + c) * L.record;
+    *reinterpret_cast<uint16_t*>(rec + L.scales + 256 * gg + 2 * nl) = scales[idx];
+    if (zeros && (nl & 7) == 0)
+        *reinterpret_cast<int32_t*>(rec + L.zeros + 64 * gg + 4 * (nl / 8)) = zeros[(size_t)gi * (N / 8) + n / 8];
 }
 
 }  // namespace
 
 int launch_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
                   int group, int sym, void* tiled, cudaStream_t stream) {
-    const TiledOffsets off = tiled_offsets(K, N, group, sym);
-    const size_t total = (size_t)(K / 8) * N;
+    const TiledLayout L = tiled_layout(K, N, group, sym);
     const int threads = 256;
-    repack_codes_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(
-        codes, K, N, sym, static_cast<int32_t*>(tiled));
+    const size_t words = (size_t)(K / 8) * N;
+    repack_codes_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, stream>>>(
+        codes, K, N, sym, L.record, static_cast<uint8_t*>(tiled));
     if (cudaGetLastError() != cudaSuccess) return W4A16_ECUDA;
-    char* base = static_cast<char*>(tiled);
-    if (cudaMemcpyAsync(base + off.scales, scales, off.scales_bytes, cudaMemcpyDeviceToDevice,
-                        stream) != cudaSuccess)
-        return W4A16_ECUDA;
-    if (!sym && cudaMemcpyAsync(base + off.zeros, zeros, off.zeros_bytes, cudaMemcpyDeviceToDevice,
-                                stream) != cudaSuccess)
-        return W4A16_ECUDA;
-    return W4A16_OK;
+    const size_t meta = (size_t)(K / group) * N;
+    repack_meta_kernel<<<(unsigned)((meta + threads - 1) / threads), threads, 0, stream>>>(
+        static_cast<const uint16_t*>(scales), sym ? nullptr : zeros, K, N, group, L, static_cast<uint8_t*>(tiled));
+    return launch_status();
 }
 
 }  // namespace w4a16

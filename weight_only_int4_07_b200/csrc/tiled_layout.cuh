@@ -1,4 +1,20 @@
-// tiled_layout.cuh -- index map and region offsets of the tiled weight buffer (w4a16_repack).
+// tiled_layout.cuh -- the tiled weight buffer of w4a16_repack: one contiguous record per unit of
+// 128 output channels x 128 input channels.
+//
+// "INT4 and Low-Bit Inference", section 5 "The kernel is half the story": weights are permuted once
+// at load so that unpacking is branch-free and the reads are coalesced; "4.3 Weight-only INT4",
+// section 4: a pre-reordered layout that suits runtime reads. The form is the library's own:
+//   unit (t, c) = channels [128 t, 128 t + 128) x input channels [128 c, 128 c + 128), record index
+//   t * (K / 128) + c, R = 8192 + G * 256 + (asym ? G * 64 : 0) bytes, G = 128 / group;
+//   codes  [0, 8192): block h = 0..3 (input channels 128 c + 32 h ..) at 2048 h; channel n owns the
+//          16 bytes at slot (n ^ 2h) of its block; word w of them is packed row 16 c + 4 h + w,
+//          nibbles re-ordered (slot p <- element 2p, slot p + 4 <- element 2p + 1), symmetric
+//          codes offset-binary (q + 8);
+//   scales [8192, + G * 256): group gg of the unit at 256 gg, channel n at + 2 n;
+//   zeros  (asymmetric) [8192 + G * 256, + G * 64): group gg at 64 gg, the tile's 16 plain words.
+// A CTA that streams consecutive units reads one contiguous range (one bulk copy per stage); the
+// XOR slot makes the 16-byte reads of an MMA fragment (lanes g, t reading block t, channel g)
+// bank-conflict free.
 #pragma once
 
 #include <stddef.h>
@@ -6,15 +22,32 @@
 
 namespace w4a16 {
 
-constexpr int kTileN = 128;        // output channels per tile
-constexpr int kTileK = 64;         // input channels per tile (8 packed rows)
-constexpr int kTileWords = 1024;   // 128 x 8 int32 words = 4 KiB
+constexpr int kTileN = 128;   // output channels per unit
+constexpr int kTileK = 128;   // input channels per unit (16 packed rows)
 
-// Word offset of plain word (j, n) inside the tiled codes region.
-__host__ __device__ __forceinline__ size_t tiled_word_offset(int j, int n, int K) {
-    const int t = n / kTileN, c = j / 8, jl = j % 8, nl = n % kTileN;
-    const size_t tile = (size_t)t * (K / kTileK) + c;
-    return tile * kTileWords + (size_t)((jl / 4) * 512 + nl * 4 + (jl % 4));
+struct TiledLayout {
+    uint32_t record;   // bytes per unit record
+    uint32_t scales;   // scales offset inside a record
+    uint32_t zeros;    // zeros offset inside a record
+    int groups;        // groups of K per unit
+    size_t total;      // whole buffer
+};
+
+__host__ __device__ __forceinline__ TiledLayout tiled_layout(int K, int N, int group, int sym) {
+    TiledLayout l;
+    l.groups = 128 / group;
+    l.scales = 8192u;
+    l.zeros = 8192u + 256u * (uint32_t)l.groups;
+    l.record = l.zeros + (sym ? 0u : 64u * (uint32_t)l.groups);
+    l.total = (size_t)(N / kTileN) * (size_t)(K / kTileK) * l.record;
+    return l;
+}
+
+// Byte offset of plain word (j, n) (packed row j, channel n) in the tiled buffer.
+__host__ __device__ __forceinline__ size_t tiled_word_byte(int j, int n, int K, uint32_t record) {
+    const int t = n / kTileN, nl = n % kTileN, c = j / 16, h = (j % 16) / 4, w = j % 4;
+    const size_t rec = (size_t)t * (K / kTileK) + c;
+    return rec * record + (size_t)(2048 * h + 16 * (nl ^ (2 * h)) + 4 * w);
 }
 
 // Re-encoding of one plain word (nibble i = element i) for the tiled layout: slot p <- element
@@ -29,27 +62,6 @@ __host__ __device__ __forceinline__ uint32_t tiled_encode_word(uint32_t w, int s
         t |= ((w >> (8 * p + 4)) & 0xFu) << (16 + 4 * p);    // element 2p + 1
     }
     return t;
-}
-
-struct TiledOffsets {
-    size_t codes, codes_bytes;
-    size_t scales, scales_bytes;
-    size_t zeros, zeros_bytes;
-    size_t total;
-};
-
-__host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-__host__ __device__ __forceinline__ TiledOffsets tiled_offsets(int K, int N, int group, int sym) {
-    TiledOffsets o;
-    o.codes = 0;
-    o.codes_bytes = (size_t)K * N / 2;
-    o.scales = align256(o.codes_bytes);
-    o.scales_bytes = (size_t)(K / group) * N * 2;
-    o.zeros = align256(o.scales + o.scales_bytes);
-    o.zeros_bytes = sym ? 0 : (size_t)(K / group) * (N / 8) * 4;
-    o.total = align256(o.zeros + o.zeros_bytes);
-    return o;
 }
 
 }  // namespace w4a16

@@ -29,7 +29,6 @@ LAYOUT_TILED = 1
 KERNEL_AUTO = 0
 KERNEL_GEMV = 1
 KERNEL_TC = 2
-KERNEL_SKINNY = 3
 
 _DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
 _TORCH_DTYPES = {F16: torch.float16, BF16: torch.bfloat16}
