@@ -8,9 +8,11 @@
 // Work split. The weights are the tiled buffer's unit records (128 channels x 128 K, codes then
 // scales then zeros), ordered tile-major, so a contiguous range of units is one contiguous range
 // of bytes. One CTA per SM takes floor(U / P) or ceil(U / P) consecutive units. A tile whose units
-// all belong to one CTA is written straight to C; a tile cut between CTAs is finished by the last
-// of them to arrive (a counter per tile in the workspace), which adds the FP32 partial sums of
-// all of them in CTA order, so the result does not depend on timing.
+// all belong to one CTA is written straight to C. A tile cut between CTAs cf < ... < cl is the
+// last tile of cf's range and the first of every later one: each later CTA publishes its FP32
+// sums to the workspace and counts them (release, no wait) as soon as it has them; cf, at the end
+// of its range, waits for the count (acquire, bounded), adds the sums in CTA order, writes C and
+// resets the counter. The result does not depend on timing.
 //
 // Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each;
 // the last warp to leave a stage refills it with the stage ns positions later, so no warp waits
@@ -173,7 +175,7 @@ struct GsParams {
     const uint8_t* tiled;
     void* C;
     int* counters;      // one int per tile, zero between calls
-    float* partials;    // [P][2][M][128]
+    float* partials;    // [P][M][128]: sums a CTA publishes for the tile that opens its range
     int* dev_status;
     int M, K, N, sym, ns, P;
     uint32_t record, scales_off, zeros_off;
@@ -204,7 +206,6 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     uint64_t* empty = full + ns;
     int* flags = reinterpret_cast<int*>(empty + ns);
     volatile int* abort_flag = flags;
-    volatile int* last_flag = flags + 1;
     int* issued = flags + 2;            // [ns] copies issued into each slot
     int* leave = flags + 2 + ns;        // [ns] warps that have left the slot's current stage
 
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
             const size_t n0 = (size_t)tile * 128;
             const int cf = unit_owner((long long)tile * steps, U, P);
             const int cl = unit_owner((long long)tile * steps + steps - 1, U, P);
-            float* part = p.partials + ((size_t)cta * 2 + (tile == (int)(u0 / steps) ? 0 : 1)) * (size_t)M * 128;
+            float vals[2][NB][4];
 #pragma unroll
             for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
@@ -330,34 +331,69 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                        if (m < M) {
-                            const float v = tot[rt][b][e] + rb[m * 128 + ch] + rb[(M + m) * 128 + ch] +
-                                            rb[(2 * M + m) * 128 + ch];
-                            if (cf == cl) C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(v);
-                            else part[m * 128 + ch] = v;
-                        }
+                        vals[rt][b][e] = m < M ? tot[rt][b][e] + rb[m * 128 + ch] + rb[(M + m) * 128 + ch] +
+                                                     rb[(2 * M + m) * 128 + ch]
+                                               : 0.0f;
                     }
-            if (cf != cl) {
-                // the last CTA of the tile to arrive adds every CTA's partial sums in CTA order
-                named_bar(2, 32 * kGsGroupWarps);
-                if (threadIdx.x == 0) {
-                    int old;
-                    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + tile)
-                                 : "memory");
-                    *last_flag = (old == cl - cf) ? 1 : 0;
-                }
-                named_bar(2, 32 * kGsGroupWarps);
-                if (*last_flag) {
-                    for (int e = threadIdx.x; e < M * 128; e += 32 * kGsGroupWarps) {
-                        float sum = 0.0f;
-                        for (int c = cf; c <= cl; ++c) {
-                            const int sl = (tile == (int)(unit_begin(c, U, P) / steps)) ? 0 : 1;
-                            sum += __ldcg(p.partials + ((size_t)c * 2 + sl) * (size_t)M * 128 + e);
+            if (cf == cl || cta == cf) {
+                if (cf != cl) {
+                    // the tile is cut between CTAs cf .. cl and this is cf: the tile is the last of
+                    // its range. Wait until every later CTA of the tile has published its sums (they
+                    // hold the tile at the start of their ranges), then add them in CTA order.
+                    if (threadIdx.x == 0) {
+                        const uint64_t t0 = globaltimer_ns();
+                        for (;;) {
+                            int n;
+                            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + tile)
+                                         : "memory");
+                            if (n >= cl - cf) break;
+                            if (*abort_flag || globaltimer_ns() - t0 > kGsSpin) {
+                                *abort_flag = 1;
+                                report_status(p.dev_status, W4A16_ETIMEOUT);
+                                break;
+                            }
                         }
-                        C[(size_t)(e >> 7) * N + n0 + (e & 127)] = Act<T>::from_f32(sum);
+                        p.counters[tile] = 0;
                     }
-                    if (threadIdx.x == 0) p.counters[tile] = 0;
+                    named_bar(2, 32 * kGsGroupWarps);
+                    for (int c = cf + 1; c <= cl; ++c) {
+                        const float* part = p.partials + (size_t)c * M * 128;
+#pragma unroll
+                        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                                    if (m < M) vals[rt][b][e] += __ldcg(part + m * 128 + ch);
+                                }
+                    }
                 }
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                            if (m < M) C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(vals[rt][b][e]);
+                        }
+            } else {
+                // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
+                // count them, without waiting
+                float* part = p.partials + (size_t)cta * M * 128;
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                            if (m < M) part[m * 128 + ch] = vals[rt][b][e];
+                        }
+                named_bar(2, 32 * kGsGroupWarps);
+                if (threadIdx.x == 0)
+                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + tile) : "memory");
             }
         }
         zero_tot();
@@ -556,7 +592,7 @@ GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_s
     pl.smem = fixed + ns * pl.stage_bytes;
     const long long total_units = (long long)(N / 128) * (K / 128);
     pl.ctas = n_sm > 0 ? (int)(total_units < n_sm ? total_units : n_sm) : 0;
-    pl.partial_bytes = (size_t)(n_sm > 0 ? n_sm : 0) * 2 * M * 128 * 4;
+    pl.partial_bytes = (size_t)(n_sm > 0 ? n_sm : 0) * M * 128 * 4;
     pl.ok = pl.ctas > 0;
     return pl;
 }
