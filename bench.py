@@ -36,10 +36,19 @@ if ROOT not in sys.path:
 LLAMA8B_LINEARS = (("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672),
                    ("down", 14336, 4096))
 LAYERS = 32
+LLAMA70B_LINEARS = (("qkv", 8192, 10240), ("o", 8192, 8192), ("gate_up", 8192, 57344),
+                    ("down", 28672, 8192))
+LAYERS_70B = 80
 GROUP = 128
 SYM = 0
 SWEEP_K, SWEEP_N, SWEEP_M = 8192, 28672, 256
 METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=256, as % of B200 roofline"
+# DRAM traffic (read + write) per algorithmic byte of the decode kernel, from one ncu capture of
+# the same kernel on a layer larger than L2 (profiles/gemv_stream_gate_up70b_m1.md): every unit
+# record streams once, so traffic scales with the units a launch processes.
+DECODE_TRAFFIC_RATIO = 1.016
+DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of gemv_stream_kernel "
+                         "(fp16, M=1) on the 8192x57344 layer, scaled by bytes per launch")
 
 
 # ----------------------------------------------------------------------------- work model
@@ -161,15 +170,18 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 class DecodeStack:
-    """Quantized Llama-3-8B-shaped linears, LAYERS copies, plus per-GEMM activations/outputs."""
+    """Quantized decode linears (Llama-3-8B-shaped by default), `layers` copies of each, plus
+    per-GEMM activations (fp16 or bf16) and outputs."""
 
-    def __init__(self, torch, native, synthetic, seed, layers=LAYERS, M=1):
+    def __init__(self, torch, native, synthetic, seed, layers=LAYERS, M=1, linears=LLAMA8B_LINEARS,
+                 bf16=False):
         self.torch, self.native = torch, native
         dev = torch.device("cuda")
         self.M = M
         self.layers = []
         uniq = []
-        for i, (name, K, N) in enumerate(LLAMA8B_LINEARS):
+        tdt = torch.bfloat16 if bf16 else torch.float16
+        for i, (name, K, N) in enumerate(linears):
             Wb = synthetic.weights_normal(K, N, seed + i)
             W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).to(dev)
             codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
@@ -190,14 +202,15 @@ class DecodeStack:
             self.layers.append(lay)
         del uniq
         # activations: one flat device buffer (and a pinned host twin for the e2e leg)
-        self.a_elems = sum(M * K for (_, K, _) in LLAMA8B_LINEARS) * layers
-        self.c_elems = sum(M * N for (_, _, N) in LLAMA8B_LINEARS) * layers
-        Ab = synthetic.activations(1, self.a_elems, seed + 100)
-        self.A_host = torch.from_numpy(Ab.view(np.int16).reshape(-1)).view(torch.float16).pin_memory()
+        self.a_elems = sum(M * K for (_, K, _) in linears) * layers
+        self.c_elems = sum(M * N for (_, _, N) in linears) * layers
+        Ab = synthetic.activations(1, self.a_elems, seed + 100,
+                                   dtype=synthetic.BF16 if bf16 else synthetic.F16)
+        self.A_host = torch.from_numpy(Ab.view(np.int16).reshape(-1)).view(tdt).pin_memory()
         self.A = self.A_host.to(dev)
-        self.C = torch.empty(self.c_elems, dtype=torch.float16, device=dev)
-        self.C_host = torch.empty(self.c_elems, dtype=torch.float16).pin_memory()
-        ws = max(native.w4a16_workspace_bytes(M, N, K, GROUP) for (_, K, N) in LLAMA8B_LINEARS)
+        self.C = torch.empty(self.c_elems, dtype=tdt, device=dev)
+        self.C_host = torch.empty(self.c_elems, dtype=tdt).pin_memory()
+        ws = max(native.w4a16_workspace_bytes(M, N, K, GROUP) for (_, K, N) in linears)
         self.ws = torch.zeros(max(ws, 16), dtype=torch.uint8, device=dev)
         # views per GEMM
         self.calls = []
@@ -331,6 +344,36 @@ def time_e2e(torch, stack, steps, warmup):
     end.record()
     torch.cuda.synchronize()
     return start.elapsed_time(end) / steps
+
+
+def bench_70b(torch, native, synthetic, seed, steps, warmup, rank):
+    """GB/s of one M = 1 decode step over a Llama-3-70B-shaped linear stack: 80 layers x (qkv, o,
+    gate+up, down), g128 asymmetric INT4, bf16 activations, 35 GB of packed weights, replayed from
+    a CUDA graph; plus each shape's mean device time per launch."""
+    stack = DecodeStack(torch, native, synthetic, seed, layers=LAYERS_70B, linears=LLAMA70B_LINEARS,
+                        bf16=True)
+    for _ in range(max(warmup, 1)):
+        stack.step()
+    torch.cuda.synchronize()
+    graph = new_graph(torch)
+    with torch.cuda.graph(graph):
+        stack.step()
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        graph.replay()
+    with ClockSampler(rank) as clk:
+        ms = time_graph(torch, graph, steps, 1, None)
+    launches = time_per_launch(torch, stack, 1)
+    per_shape = {name: {"K": K, "N": N, "mean_us": 1e3 * statistics.mean(v),
+                        "gbs": algorithmic_bytes(1, K, N) / (statistics.mean(v) * 1e-3) / 1e9}
+                 for (name, K, N), v in launches.items()}
+    out = {"ms_per_step": ms, "bytes_per_step": stack.bytes_per_step,
+           "weight_bytes_per_step": stack.weight_bytes, "gemms_per_step": len(stack.calls),
+           "per_shape": per_shape, "clocks": clk.summary()}
+    del graph, stack
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
@@ -528,8 +571,10 @@ def run_ours(args):
                  for (name, K, N), v in launches.items()}
     achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
     kernel = native.w4a16_select_kernel(1, 4096, 4096, GROUP)
+    traffic = DECODE_TRAFFIC_RATIO * tot_bytes / n_launch if stack.tiled else None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "traffic_source": DECODE_TRAFFIC_SOURCE if traffic else None,
                 "kernel": {1: "gemv", 2: "tc"}.get(kernel, str(kernel)),
                 "bytes_per_launch": tot_bytes / n_launch, "launch_us": 1e3 * tot_ms / n_launch,
                 "peak_source": peaks["source"], "per_shape": per_shape}
@@ -548,11 +593,29 @@ def run_ours(args):
     weight_bytes = stack.weight_bytes
     bytes_per_step = stack.bytes_per_step
 
+    del stack
+    torch.cuda.empty_cache()
+
+    # the same metric over the 70B-shaped stack (the layers the ">= 75% of HBM" target names)
+    m1_70b = None
+    if not args.skip_70b:
+        r70 = bench_70b(torch, native, synthetic, replica_seed(7000, rank), max(2, min(args.steps, 10)),
+                        args.warmup, local_rank)
+        ms70 = max_over_ranks(r70["ms_per_step"], world, dev)
+        gbs70 = world * r70["bytes_per_step"] / (ms70 * 1e-3) / 1e9
+        m1_70b = {"value": gbs70, "unit": "GB/s", "ms_per_step": ms70,
+                  "frac": gbs70 / world / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                  "peak_source": peaks["source"], "per_shape": r70["per_shape"], "clocks": r70["clocks"],
+                  "config": {"workload": "llama3-70b decode linears (qkv 8192x10240, o 8192x8192, "
+                                         "gate+up 8192x57344, down 28672x8192), M=1, g128 asym INT4, "
+                                         "bf16 acts, 80 layers per step",
+                             "gemms_per_step": r70["gemms_per_step"],
+                             "weight_bytes_per_step": r70["weight_bytes_per_step"],
+                             "algorithmic_bytes_per_step": r70["bytes_per_step"]}}
+
     # M = 256 on the sweep layer (TFLOPS)
     m256 = None
     if not args.skip_m256:
-        del stack
-        torch.cuda.empty_cache()
         r = bench_m256(torch, native, synthetic, replica_seed(5000, rank), max(2, min(args.steps, 10)),
                        args.warmup)
         ms256 = max_over_ranks(r["ms"], world, dev)
@@ -590,12 +653,41 @@ def run_ours(args):
                            "timing": "CUDA graph replay of one step, CUDA events"},
                 "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
                 "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
-                "m256": m256}
+                "m1_70b": m1_70b, "m256": m256}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_single(args):
+    """A few launches of one tiled W4A16 GEMM (the small case profiled under ncu): weights of
+    (K, N) on two rotating copies, M rows of activations; prints one line, times nothing."""
+    import torch
+
+    from weight_only_int4_07_b200 import build, native, synthetic
+
+    K, N, M = (int(x) for x in args.single.split(","))
+    torch.cuda.set_device(0)
+    build.build()
+    bf16 = args.dtype == "bf16"
+    Wb = synthetic.weights_normal(K, N, 3)
+    W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
+    codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
+    del W
+    copies = [native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM) for _ in range(2)]
+    Ab = synthetic.activations(M, K, 4, dtype=synthetic.BF16 if bf16 else synthetic.F16)
+    A = torch.from_numpy(Ab.view(np.int16)).view(torch.bfloat16 if bf16 else torch.float16).cuda()
+    C = torch.empty((M, N), dtype=A.dtype, device="cuda")
+    ws = torch.zeros(max(native.w4a16_workspace_bytes(M, N, K, GROUP), 16), dtype=torch.uint8, device="cuda")
+    for i in range(args.launches):
+        native.w4a16_gemm(A, copies[i % 2], None, None, N, GROUP, SYM, layout=native.LAYOUT_TILED, C=C,
+                          workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"single": [K, N, M], "dtype": args.dtype, "launches": args.launches,
+                      "kernel": {1: "gemv", 2: "tc"}[native.w4a16_select_kernel(M, N, K, GROUP)]}))
     return 0
 
 
@@ -606,9 +698,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--skip-m256", action="store_true")
+    ap.add_argument("--skip-70b", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--single", default=None, help="K,N,M: a few launches of one GEMM, untimed")
+    ap.add_argument("--dtype", choices=("f16", "bf16"), default="f16")
+    ap.add_argument("--launches", type=int, default=4)
     args = ap.parse_args(argv)
+    if args.single:
+        return run_single(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
