@@ -430,6 +430,74 @@ def bench_m256(torch, native, synthetic, seed, steps, warmup, copies=4):
             "layout": "tiled" if use_tiled else "plain"}
 
 
+def bench_naive(torch, native, synthetic, seed, steps, warmup, copies=4):
+    """The naive path the fused kernels are measured against: the packed weight expanded to a
+    16-bit matrix by the library's dequantize kernel, then the library GEMM (torch.matmul, FP32
+    accumulation). Per shape (the four Llama-3-8B decode linears at M = 1 with fp16 activations,
+    and the sweep layer at M = 256 with bf16 activations) the mean device time of each half,
+    rotating `copies` packed weight copies. GB/s counts the same algorithmic bytes as the fused
+    path, so the two are directly comparable."""
+    dev = torch.device("cuda")
+    prev = (torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction,
+            torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction)
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = False
+    shapes = [(name, K, N, 1, torch.float16, synthetic.F16) for (name, K, N) in LLAMA8B_LINEARS]
+    shapes.append(("sweep_m256", SWEEP_K, SWEEP_N, SWEEP_M, torch.bfloat16, synthetic.BF16))
+    stream = torch.cuda.current_stream()
+    out = {}
+    try:
+        for i, (name, K, N, M, tdt, sdt) in enumerate(shapes):
+            Wb = synthetic.weights_normal(K, N, seed + i)
+            W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).to(dev)
+            codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
+            del W
+            mats = [(codes.clone(), scales.clone(), None if zeros is None else zeros.clone())
+                    for _ in range(copies)]
+            del codes, scales, zeros
+            Ab = synthetic.activations(M, K, seed + 50 + i, dtype=sdt)
+            A = torch.from_numpy(Ab.view(np.int16)).view(tdt).to(dev)
+            Wd = torch.empty((K, N), dtype=tdt, device=dev)
+            C = torch.empty((M, N), dtype=tdt, device=dev)
+
+            def run(j, evs=None):
+                c, sc, z = mats[j % copies]
+                if evs:
+                    evs[0].record(stream)
+                native.w4a16_dequantize(c, sc, z, K, N, GROUP, SYM, out=Wd)
+                if evs:
+                    evs[1].record(stream)
+                torch.matmul(A, Wd, out=C)
+                if evs:
+                    evs[2].record(stream)
+
+            for j in range(max(warmup, 1)):
+                run(j)
+            torch.cuda.synchronize()
+            torch.cuda._sleep(int(20e6))
+            rec = []
+            for j in range(steps * copies):
+                evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                run(j, evs)
+                rec.append(evs)
+            torch.cuda.synchronize()
+            deq = statistics.mean(e[0].elapsed_time(e[1]) for e in rec)
+            mm = statistics.mean(e[1].elapsed_time(e[2]) for e in rec)
+            tot = deq + mm
+            out[name] = {"K": K, "N": N, "M": M, "acts": "fp16" if tdt == torch.float16 else "bf16",
+                         "dequant_us": 1e3 * deq, "gemm_us": 1e3 * mm, "total_us": 1e3 * tot,
+                         "gbs": algorithmic_bytes(M, K, N) / (tot * 1e-3) / 1e9,
+                         "tflops": gemm_flops(M, K, N) / (tot * 1e-3) / 1e12,
+                         "dequant_gbs": (algorithmic_bytes(0, K, N, out_bytes=0) + 2 * K * N)
+                         / (deq * 1e-3) / 1e9}
+            del mats, A, Wd, C
+            torch.cuda.empty_cache()
+    finally:
+        (torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction,
+         torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction) = prev
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def host_cores():
     try:
@@ -629,6 +697,17 @@ def run_ours(args):
                            "acts": "bf16", "weights": "N(0,0.02) with 0.1% outliers x20",
                            "l2": "4 rotating weight copies of 122 MB"}}
 
+    # the naive path (dequantize to 16 bits, then the library GEMM) on the same shapes
+    naive = None
+    if not args.skip_naive:
+        naive = bench_naive(torch, native, synthetic, replica_seed(9000, rank), max(2, min(args.steps, 10)),
+                            args.warmup)
+        for name, r in naive.items():
+            fused_us = (roofline["per_shape"][name]["mean_us"] if name in roofline["per_shape"]
+                        else (1e3 * m256["ms"] if (name == "sweep_m256" and m256) else None))
+            r["fused_us"] = fused_us
+            r["fused_speedup"] = None if fused_us is None else r["total_us"] / fused_us
+
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         threads = host_cores()
@@ -653,7 +732,7 @@ def run_ours(args):
                            "timing": "CUDA graph replay of one step, CUDA events"},
                 "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
                 "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
-                "m1_70b": m1_70b, "m256": m256}
+                "m1_70b": m1_70b, "m256": m256, "naive": naive}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -700,6 +779,7 @@ def main(argv=None):
     ap.add_argument("--skip-m256", action="store_true")
     ap.add_argument("--skip-70b", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-naive", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--single", default=None, help="K,N,M: a few launches of one GEMM, untimed")
     ap.add_argument("--dtype", choices=("f16", "bf16"), default="f16")

@@ -110,6 +110,23 @@ W4A16_API int w4a16_quantize(const void* W, int K, int N, int group, int sym, in
                    int32_t* zeros, int* dev_status, void* stream);
 
 /*
+ * w4a16_dequantize -- the packed weight expanded to a 16-bit matrix: w[k, n] = (q - z) * s,
+ *   exact in FP32 and rounded once to out_dtype. This is the naive path that the fused kernels
+ *   are measured against: "4.3 Weight-only INT4", section 4 (dequantize the INT4 matrix to FP16 in
+ *   memory, then a standard GEMM: the weights cross HBM as 4 bits, then twice as 16 bits);
+ *   "INT4 and Low-Bit Inference", section 5 "The kernel is half the story".
+ * Arguments
+ *   codes, scales, zeros  device, plain layout as produced by w4a16_quantize (zeros NULL iff sym).
+ *   K, N, group, sym      as for w4a16_quantize.
+ *   out_dtype             W4A16_F16 or W4A16_BF16.
+ *   W                     device out, [K, N] row-major, out_dtype (2 K N bytes).
+ *   stream                cudaStream_t.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED or W4A16_ECUDA.
+ */
+W4A16_API int w4a16_dequantize(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
+                     int group, int sym, int out_dtype, void* W, void* stream);
+
+/*
  * w4a16_repack_bytes -- size in bytes of the tiled buffer for a K x N weight (0 on bad shape).
  */
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);

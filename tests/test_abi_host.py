@@ -37,7 +37,8 @@ def L():
 def test_headers_declare_the_entry_points():
     names = _declared_symbols()
     for required in ("w4a16_quantize", "w4a16_gemm", "w4a16_repack", "w4a16_repack_bytes",
-                     "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str"):
+                     "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str",
+                     "w4a16_dequantize"):
         assert required in names
 
 
@@ -147,3 +148,21 @@ def test_repack_rejects_bad_arguments(L):
     assert r(A16, B16, None, 256, 128, 128, 0, D16, None) == native.EINVAL
     assert r(A16, B16, C16, 256, 128, 128, 1, D16, None) == native.EINVAL
     assert r(A16, B16, C16, 256, 128, 128, 0, MIS, None) == native.EALIGN
+
+
+def test_dequantize_rejects_bad_arguments_before_any_launch(L):
+    P = ctypes.c_void_p
+    ok = dict(codes=P(1 << 20), scales=P(2 << 20), zeros=P(3 << 20), K=256, N=128, group=128, sym=0,
+              dt=native.F16, W=P(4 << 20))
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.w4a16_dequantize(a["codes"], a["scales"], a["zeros"], a["K"], a["N"], a["group"],
+                                  a["sym"], a["dt"], a["W"], None)
+    assert call(group=48) == native.EUNSUPPORTED
+    assert call(K=100) == native.EINVAL
+    assert call(dt=7) == native.EINVAL
+    assert call(W=None) == native.EINVAL
+    assert call(sym=1) == native.EINVAL                   # zeros given for a symmetric weight
+    assert call(zeros=None) == native.EINVAL              # asymmetric without zeros
+    assert call(W=P((4 << 20) + 8)) == native.EALIGN

@@ -498,3 +498,39 @@ def test_gemm_auto_sweep_shape_sampled_skinny(M):
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+# ----------------------------------------------------------------------------- naive path
+@pytest.mark.parametrize("sym,group,a_dtype,K,N", [(0, 128, 0, 1024, 384), (1, 128, 1, 1024, 384),
+                                                   (0, 32, 1, 1024, 384), (1, 64, 0, 1024, 384),
+                                                   (0, 64, 0, 192, 264), (0, 128, 1, 4096, 6144)])
+def test_dequantize_bit_exact(sym, group, a_dtype, K, N):
+    """The expanded 16-bit weight equals the oracle's FP64 (q - z) * s rounded once (N = 264: a
+    ragged last block of column groups; 4096 x 6144: the 8B qkv shape)."""
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("student_t" if sym else "normal", K, N, group, sym, 77)
+    tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
+    Wd = native.w4a16_dequantize(gc, gs, gz, K, N, group, sym, dtype=tdt)
+    torch.cuda.synchronize()
+    expect = oracle.encode16(oracle.dequant(oc, os_, oz, K, N, group, sym), a_dtype)
+    assert np.array_equal(_to_np16(Wd), expect)
+
+
+@pytest.mark.parametrize("M,a_dtype", [(1, 0), (16, 1), (256, 1)])
+def test_naive_path_within_bound(M, a_dtype):
+    """Dequantize, then the library GEMM (FP32 accumulation): the naive path of the pages, held to
+    the same bound as the fused kernels."""
+    K, N, group, sym = 2048, 1024, 128, 0
+    Wb, (oc, os_, oz), (gc, gs, gz) = _quantized("normal", K, N, group, sym, 78)
+    Ab, A = _acts(M, K, 79 + M, a_dtype)
+    prev = torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction
+    prev_bf = torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = False
+    try:
+        Wd = native.w4a16_dequantize(gc, gs, gz, K, N, group, sym, dtype=A.dtype)
+        C = torch.matmul(A, Wd)
+        torch.cuda.synchronize()
+    finally:
+        torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = prev
+        torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = prev_bf
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)

@@ -12,6 +12,7 @@ from .native import (  # noqa: F401
     LAYOUT_PLAIN,
     LAYOUT_TILED,
     W4A16Error,
+    w4a16_dequantize,
     w4a16_gemm,
     w4a16_quantize,
     w4a16_repack,

@@ -96,6 +96,20 @@ W4A16_API int w4a16_quantize(const void* W, int K, int N, int group, int sym, in
                            static_cast<cudaStream_t>(stream));
 }
 
+W4A16_API int w4a16_dequantize(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
+                               int group, int sym, int out_dtype, void* W, void* stream) {
+    int st = check_shape(K, N, group);
+    if (st != W4A16_OK) return st;
+    if (sym != 0 && sym != 1) return W4A16_EINVAL;
+    if (out_dtype != W4A16_F16 && out_dtype != W4A16_BF16) return W4A16_EINVAL;
+    if (!codes || !scales || !W) return W4A16_EINVAL;
+    if (sym ? zeros != nullptr : zeros == nullptr) return W4A16_EINVAL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(W) || (zeros && !aligned16(zeros)))
+        return W4A16_EALIGN;
+    return launch_dequantize(codes, scales, zeros, K, N, group, sym, out_dtype, W,
+                             static_cast<cudaStream_t>(stream));
+}
+
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym) {
     if (check_shape(K, N, group) != W4A16_OK || (sym != 0 && sym != 1)) return 0;
     if (N % kTileN != 0 || K % kTileK != 0) return 0;

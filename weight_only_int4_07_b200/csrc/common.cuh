@@ -46,6 +46,9 @@ inline int launch_status() {
 int launch_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes, void* scales,
                     int32_t* zeros, int* dev_status, cudaStream_t stream);
 
+int launch_dequantize(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N, int group,
+                      int sym, int out_dtype, void* W, cudaStream_t stream);
+
 int launch_repack(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N,
                   int group, int sym, void* tiled, cudaStream_t stream);
 

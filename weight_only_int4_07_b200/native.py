@@ -54,6 +54,8 @@ def lib():
     P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.w4a16_quantize.argtypes = [P, I, I, I, I, P, P, P, P, P]
     L.w4a16_quantize.restype = I
+    L.w4a16_dequantize.argtypes = [P, P, P, I, I, I, I, I, P, P]
+    L.w4a16_dequantize.restype = I
     L.w4a16_repack_bytes.argtypes = [I, I, I, I]
     L.w4a16_repack_bytes.restype = S
     L.w4a16_repack.argtypes = [P, P, P, I, I, I, I, P, P]
@@ -110,6 +112,17 @@ def w4a16_quantize(W, group, sym, codes=None, scales=None, zeros=None, dev_statu
                               _ptr(zeros), _ptr(dev_status), _stream())
     _check("w4a16_quantize", st)
     return codes, scales, (None if sym else zeros)
+
+
+def w4a16_dequantize(codes, scales, zeros, K, N, group, sym, dtype=None, out=None):
+    """The packed weight as a 16-bit [K, N] matrix, (q - z) * s rounded once (the naive path)."""
+    dtype = torch.float16 if dtype is None else dtype
+    if out is None:
+        out = torch.empty((K, N), dtype=dtype, device=codes.device)
+    st = lib().w4a16_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), K, N, group, int(sym),
+                                _DTYPES[out.dtype], _ptr(out), _stream())
+    _check("w4a16_dequantize", st)
+    return out
 
 
 def w4a16_repack_bytes(K, N, group, sym) -> int:
