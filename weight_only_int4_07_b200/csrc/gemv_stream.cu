@@ -15,8 +15,9 @@
 // resets the counter. The result does not depend on timing.
 //
 // Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each;
-// the last warp to leave a stage refills it with the stage ns positions later, so no warp waits
-// for another to issue a copy. Sixteen warps in four groups: group q takes unit q of every stage,
+// lane 0 of each warp leaving a stage counts the warp out on a shared counter, and the warp that
+// completes the count refills the slot with the stage ns positions later, so no warp waits for
+// another to issue a copy. Sixteen warps in four groups: group q takes unit q of every stage,
 // warp w of a group owns channels 32 w .. 32 w + 31 of the unit.
 //
 // Math (warp-level tensor-core MMA, m16n8k16, FP32 accumulators), per warp and unit: lane
@@ -203,8 +204,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes;                 // 320 zero bytes
     uint8_t* stages = zrow + 384;                                         // ns x stage_bytes
     uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);
-    uint64_t* empty = full + ns;
-    int* flags = reinterpret_cast<int*>(empty + ns);
+    int* flags = reinterpret_cast<int*>(full + ns);
     volatile int* abort_flag = flags;
     int* issued = flags + 2;            // [ns] copies issued into each slot
     int* leave = flags + 2 + ns;        // [ns] warps that have left the slot's current stage
@@ -212,7 +212,6 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     if (threadIdx.x == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kGsThreads);
             issued[i] = 0;
             leave[i] = 0;
         }
@@ -408,19 +407,20 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     uint32_t ph = 0;
     for (int st = 0; st < nst; ++st) {
         if (st > 0 && !aborted) {
-            // leave stage st - 1; the last warp to leave refills the slot with stage st - 1 + ns
-            mbar_arrive(&empty[s_idx]);
+            // leave stage st - 1: every read of the slot by this warp has completed (its values
+            // were consumed by the unit's MMAs), so lane 0 counts the warp out once; the warp
+            // that completes the count of 16 refills the slot with stage st - 1 + ns. No warp
+            // waits for another.
             __syncwarp();
-            bool bad = false;
-            if (lane == 0 && atomicAdd(&leave[s_idx], 1) == kGsWarps - 1) {
-                leave[s_idx] = 0;
-                const int r = st - 1;
-                if (r + ns < nst) {
-                    if (mbar_wait(&empty[s_idx], (uint32_t)(r / ns) & 1u, abort_flag, p.dev_status, kGsSpin)) issue(r + ns);
-                    else bad = true;
+            if (lane == 0) {
+                int old;
+                asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                             : "=r"(old) : "r"(smem_u32(&leave[s_idx])) : "memory");
+                if (old == kGsWarps - 1) {
+                    leave[s_idx] = 0;
+                    if (st - 1 + ns < nst) issue(st - 1 + ns);
                 }
             }
-            if (__any_sync(0xffffffffu, bad)) aborted = true;
         }
         if (++s_idx == ns) {
             s_idx = 0;
