@@ -61,13 +61,16 @@ def _acts(M, K, seed, dtype):
     return Ab, A
 
 
-def _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=None):
+def _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=None, out_rel=0.0):
+    """C within REL * sum|a w| + ABS of the oracle, element by element; out_rel * |y| more where
+    a test's rows are dominated by one term (a 16-bit output rounding alone is up to 2^-8 |y|
+    in bf16)."""
     Y, Yabs = oracle.linear(Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
     y = oracle.decode16(_to_np16(C), a_dtype)
     if cols is not None:
         y = y[:, cols]
     err = np.abs(y - Y)
-    bound = REL * Yabs + ABS
+    bound = REL * Yabs + ABS + out_rel * np.abs(Y)
     bad = err > bound
     assert not bad.any(), (f"{bad.sum()} of {bad.size} outputs outside the bound; worst ratio "
                            f"{(err / bound).max():.3f}")
@@ -473,6 +476,34 @@ def test_gemm_stream_zero_weights_give_exact_zero(a_dtype):
                                       layout=native.LAYOUT_TILED, kernel=native.KERNEL_GEMV)
                 assert torch.count_nonzero(C[:, :256]).item() == 0
                 assert torch.count_nonzero(C[:, 256:]).item() > 0
+
+
+@pytest.mark.parametrize("sym", [0, 1])
+def test_gemm_stream_bf16_rows_outside_fp16_range(sym):
+    """bf16 activations far outside the fp16 range (rows scaled by 2^40, 2^-60, and a row whose
+    largest value is 1e30), full output within the bound: at group 128 the decode kernel scales
+    each bf16 row by a power of two before its fp16 arithmetic and scales the sums back, or keeps
+    bf16 when a row spans too many binades for an exact conversion."""
+    K, N, group = 2048, 512, 128
+    Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 61)
+    g = torch.Generator().manual_seed(62)
+    A32 = torch.randn((4, K), generator=g, dtype=torch.float32)
+    A32[0] *= 2.0 ** 40
+    A32[1] *= 2.0 ** -60
+    A32[2, 77] = 1e30
+    A = A32.to(torch.bfloat16)
+    # rows 0-1 alone: each row within 31 binades of its maximum, so the fp16 arithmetic on the
+    # scaled rows; all four: row 2 spans about 100 binades, so the bf16 arithmetic
+    for m in (2, 4):
+        Am = A[:m].contiguous()
+        Ab = Am.view(torch.int16).numpy().view(np.uint16)
+        C = native.w4a16_gemm(Am.cuda(), tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                              kernel=native.KERNEL_GEMV)
+        torch.cuda.synchronize()
+        assert torch.isfinite(C.float()).all()
+        # row 2 is dominated by its 1e30 term (|y| ~ sum|a w|), where the bf16 output rounding
+        # alone reaches 2^-8 |y|, above 2e-3 sum|a w|: that rounding is added to the bound
+        _check_gemm(C, Ab, 1, oc, os_, oz, N, group, sym, out_rel=2.0 ** -8)
 
 
 @pytest.mark.parametrize("K,N", [(8192, 10240), (8192, 8192), (8192, 57344), (28672, 8192)])

@@ -35,6 +35,7 @@
 // issuing copies, still passes every CTA barrier and tile counter, and lets the copies in
 // flight land before it exits.
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -51,6 +52,7 @@ constexpr int kGsUnitsPerStage = kGsGroups;
 constexpr int kGsMinStages = 3, kGsMaxStages = 16;
 constexpr int kGsSmemMax = 227 * 1024;
 constexpr uint64_t kGsSpin = 2000000000ull;
+constexpr int kGsZrowBytes = 512;   // the zero activation block, then per-row exponent bounds
 
 __device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {   // a >> k for b = 2^(32-k)
     uint32_t r;
@@ -155,6 +157,11 @@ struct GsOps<__nv_bfloat16> {
     }
 };
 
+template <typename X>
+struct OpsTag {
+    using type = X;
+};
+
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -182,14 +189,25 @@ struct GsParams {
     uint32_t record, scales_off, zeros_off;
     uint32_t stage_bytes, row_bytes, act_bytes, red_bytes;
     GsMasks km;
+    GsMasks km_native;   // bf16 masks, for bf16 rows kept in bf16 at group 128
 };
 
 // NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
 template <int NB, typename T, int GROUP, bool ODD>
 __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    using Ops = GsOps<T>;
     constexpr bool kPost = (GROUP == 128);   // one group per unit: scale the unit's sum
+    // bf16 activations at group 128 run the fp16 arithmetic (fewer instructions per weight)
+    // whenever that is exact: each row is scaled by a power of two 2^-k that puts its largest
+    // value in [2^14, 2^15) and converted to fp16. A bf16 value whose exponent is at most 31 below
+    // the row's largest lands on an fp16 normal or on the fp16 subnormal grid with all 8 of its
+    // significant bits, so the conversion is exact; the MMAs then form the same products
+    // a * (u - z) as bf16 operands would, and the sums are multiplied back by 2^k when C is
+    // written. When some row holds a nonzero value further below its maximum, every CTA keeps
+    // the bf16 values and the bf16 arithmetic (the decision depends only on A, so all CTAs agree).
+    constexpr bool kConv = kPost && std::is_same<T, __nv_bfloat16>::value;
+    using MathT = typename std::conditional<kConv, __half, T>::type;
+    using Ops = GsOps<MathT>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int M = p.M, K = p.K, N = p.N, ns = p.ns, P = p.P;
     const int steps = K / 128;
@@ -202,7 +220,9 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     uint8_t* acts = smem_raw;                                             // [M][RS]
     float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][3][M][128]
     uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes;                 // 320 zero bytes
-    uint8_t* stages = zrow + 384;                                         // ns x stage_bytes
+    int* rowexp = reinterpret_cast<int*>(zrow + 320);                     // [16] largest exponent per row
+    int* rowmin = reinterpret_cast<int*>(zrow + 384);                     // [16] smallest nonzero one
+    uint8_t* stages = zrow + kGsZrowBytes;                                // ns x stage_bytes
     uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);
     int* flags = reinterpret_cast<int*>(full + ns);
     volatile int* abort_flag = flags;
@@ -219,6 +239,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < 96; i += kGsThreads) reinterpret_cast<uint32_t*>(zrow)[i] = 0u;
+    if (threadIdx.x < 16) rowmin[threadIdx.x] = 255;
     __syncthreads();
     grid_dependents_launch();
 
@@ -242,6 +263,8 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     const int ch0 = 32 * wg + g;     // this lane's channels: ch0 + 8 r, r = 0..3
     const T* A = static_cast<const T*>(p.A);
 
+    bool wide = false;   // kConv: some row keeps bf16 values and the bf16 arithmetic
+
     // A may be the output of the previous kernel in the stream
     grid_dependency_wait();
     {
@@ -249,7 +272,12 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         // lanes' 16-byte reads conflict free); pairs in each 16-byte chunk stored (p0, p2, p1, p3)
         // so that each MMA's two B registers are adjacent; each CTA starts at a different chunk
         const int vpr = K / 8;
-        for (int m = 0; m < M; ++m)
+        auto chunk_off = [&](int m, int c) {
+            return (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u + (uint32_t)((c >> 2) & 3) * 80u +
+                   (uint32_t)(c & 3) * 16u;
+        };
+        for (int m = 0; m < M; ++m) {
+            uint32_t emax = 0, emin = 255;   // largest, smallest nonzero biased exponent of row m
             for (int c0 = threadIdx.x; c0 < vpr; c0 += 4 * kGsThreads) {
                 uint4 vv[4];
 #pragma unroll
@@ -261,11 +289,51 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                 for (int j = 0; j < 4; ++j)
                     if (c0 + j * kGsThreads < vpr) {
                         const int c = (c0 + j * kGsThreads + cta * 64) % vpr;
-                        const uint32_t off = (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u +
-                                             (uint32_t)((c >> 2) & 3) * 80u + (uint32_t)(c & 3) * 16u;
-                        *reinterpret_cast<uint4*>(acts + off) = make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
+                        *reinterpret_cast<uint4*>(acts + chunk_off(m, c)) =
+                            make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
+                        if constexpr (kConv) {
+                            const uint32_t x[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const uint32_t e0 = (x[q] >> 7) & 0xFFu, e1 = (x[q] >> 23) & 0xFFu;
+                                emax = max(emax, max(e0, e1));
+                                if (x[q] & 0x7FFFu) emin = min(emin, e0);
+                                if (x[q] & 0x7FFF0000u) emin = min(emin, e1);
+                            }
+                        }
                     }
             }
+            if constexpr (kConv) {
+                emax = __reduce_max_sync(0xffffffffu, emax);
+                emin = __reduce_min_sync(0xffffffffu, emin);
+                if (lane == 0) {
+                    atomicMax(&rowexp[m], (int)emax);
+                    atomicMin(&rowmin[m], (int)emin);
+                }
+            }
+        }
+        if constexpr (kConv) {
+            // second pass, in shared memory: bf16 -> 2^-k * a in fp16, unless some row is too wide
+            __syncthreads();
+            for (int m = 0; m < M; ++m) wide = wide || rowexp[m] - rowmin[m] > 31;
+            for (int m = 0; m < M && !wide; ++m) {
+                const int k = min(max(rowexp[m] - 141, -100), 114);
+                const float down = __int_as_float((127 - k) << 23);
+                for (int c0 = threadIdx.x; c0 < vpr; c0 += kGsThreads) {
+                    const int c = (c0 + cta * 64) % vpr;
+                    uint4* q = reinterpret_cast<uint4*>(acts + chunk_off(m, c));
+                    uint4 v = *q;
+                    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16) * down,
+                                                      __uint_as_float(w[i] & 0xFFFF0000u) * down);
+                        w[i] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    *q = v;
+                }
+            }
+        }
     }
     __syncthreads();
 
@@ -375,7 +443,12 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                            if (m < M) C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(vals[rt][b][e]);
+                            if (m < M) {
+                                float y = vals[rt][b][e];
+                                if constexpr (kConv)   // undo the row's 2^-k
+                                    if (!wide) y *= __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
+                                C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(y);
+                            }
                         }
             } else {
                 // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
@@ -400,6 +473,69 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         sp_lo = 0;
         seg_lo = seg_hi;
         seg_hi = seg_lo + steps < nunits ? seg_lo + steps : nunits;
+    };
+
+    // the MMAs of one unit, with the operand arithmetic of O (fp16 or bf16)
+    auto unit_math = [&](auto tag, const GsMasks& kx, const uint4 (&cw)[4], const uint16_t (&sb)[4],
+                         const uint4& zw, const uint4 (&v)[NB][4]) {
+        using O = typename decltype(tag)::type;
+        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
+            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
+            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+            const uint32_t z0 = (zws[2 * rt] >> zsh) & 0xFu, z1 = (zws[2 * rt + 1] >> zsh) & 0xFu;
+            const uint32_t za0 = O::zz_a(z0), za1 = O::zz_a(z1), zb0 = O::zz_b(z0), zb1 = O::zz_b(z1);
+            typename O::Scale sc0, sc1;
+            if constexpr (!kPost) {
+                sc0.set(sb[2 * rt]);
+                sc1.set(sb[2 * rt + 1]);
+            }
+            float acc[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t q0[4], q1[4];
+                O::unpack(w0[i], kx, q0);
+                O::unpack(w1[i], kx, q1);
+                q0[0] = O::sub_a(q0[0], za0);
+                q0[2] = O::sub_a(q0[2], za0);
+                q0[1] = O::sub_b(q0[1], zb0);
+                q0[3] = O::sub_b(q0[3], zb0);
+                q1[0] = O::sub_a(q1[0], za1);
+                q1[2] = O::sub_a(q1[2], za1);
+                q1[1] = O::sub_b(q1[1], zb1);
+                q1[3] = O::sub_b(q1[3], zb1);
+                if constexpr (!kPost) {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        q0[x] = sc0.apply(q0[x]);
+                        q1[x] = sc1.apply(q1[x]);
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    float (&d)[4] = kPost ? acc[b] : tot[rt][b];
+                    O::mma(d, q0[0], q1[0], q0[2], q1[2], v[b][i].x, v[b][i].y);
+                    O::mma(d, q0[1], q1[1], q0[3], q1[3], v[b][i].z, v[b][i].w);
+                }
+            }
+            if constexpr (kPost) {
+                const float s0 = __half2float(__ushort_as_half(sb[2 * rt]));
+                const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1]));
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    tot[rt][b][0] = fmaf(s0, acc[b][0], tot[rt][b][0]);
+                    tot[rt][b][2] = fmaf(s1, acc[b][2], tot[rt][b][2]);
+                    if (ODD) {
+                        tot[rt][b][1] = fmaf(s0, acc[b][1], tot[rt][b][1]);
+                        tot[rt][b][3] = fmaf(s1, acc[b][3], tot[rt][b][3]);
+                    }
+                }
+            }
+        }
     };
 
     bool aborted = false;
@@ -448,62 +584,11 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
             for (int i = 0; i < 4; ++i) v[b][i] = *reinterpret_cast<const uint4*>(a + 16 * i);
         }
-        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
-#pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
-            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
-            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
-            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
-            const uint32_t z0 = (zws[2 * rt] >> zsh) & 0xFu, z1 = (zws[2 * rt + 1] >> zsh) & 0xFu;
-            const uint32_t za0 = Ops::zz_a(z0), za1 = Ops::zz_a(z1), zb0 = Ops::zz_b(z0), zb1 = Ops::zz_b(z1);
-            typename Ops::Scale sc0, sc1;
-            if constexpr (!kPost) {
-                sc0.set(sb[2 * rt]);
-                sc1.set(sb[2 * rt + 1]);
-            }
-            float acc[NB][4];
-#pragma unroll
-            for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t q0[4], q1[4];
-                Ops::unpack(w0[i], km, q0);
-                Ops::unpack(w1[i], km, q1);
-                q0[0] = Ops::sub_a(q0[0], za0);
-                q0[2] = Ops::sub_a(q0[2], za0);
-                q0[1] = Ops::sub_b(q0[1], zb0);
-                q0[3] = Ops::sub_b(q0[3], zb0);
-                q1[0] = Ops::sub_a(q1[0], za1);
-                q1[2] = Ops::sub_a(q1[2], za1);
-                q1[1] = Ops::sub_b(q1[1], zb1);
-                q1[3] = Ops::sub_b(q1[3], zb1);
-                if constexpr (!kPost) {
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        q0[x] = sc0.apply(q0[x]);
-                        q1[x] = sc1.apply(q1[x]);
-                    }
-                }
-#pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    float (&d)[4] = kPost ? acc[b] : tot[rt][b];
-                    Ops::mma(d, q0[0], q1[0], q0[2], q1[2], v[b][i].x, v[b][i].y);
-                    Ops::mma(d, q0[1], q1[1], q0[3], q1[3], v[b][i].z, v[b][i].w);
-                }
-            }
-            if constexpr (kPost) {
-                const float s0 = __half2float(__ushort_as_half(sb[2 * rt]));
-                const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1]));
-#pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    tot[rt][b][0] = fmaf(s0, acc[b][0], tot[rt][b][0]);
-                    tot[rt][b][2] = fmaf(s1, acc[b][2], tot[rt][b][2]);
-                    if (ODD) {
-                        tot[rt][b][1] = fmaf(s0, acc[b][1], tot[rt][b][1]);
-                        tot[rt][b][3] = fmaf(s1, acc[b][3], tot[rt][b][3]);
-                    }
-                }
-            }
+        if constexpr (kConv) {
+            if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
+            else unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
+        } else {
+            unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
         }
     }
     while (seg_lo < nunits) emit();
@@ -583,7 +668,7 @@ GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_s
     pl.red_bytes = (size_t)2 * 3 * M * 128 * 4;
     pl.stage_bytes = ((size_t)kGsUnitsPerStage * L.record + 127) & ~(size_t)127;
     const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 8 + 8 * kGsMaxStages + 127) & ~(size_t)127;
-    const size_t fixed = pl.act_bytes + pl.red_bytes + 384 + flags;
+    const size_t fixed = pl.act_bytes + pl.red_bytes + kGsZrowBytes + flags;
     if (fixed >= (size_t)kGsSmemMax) return pl;
     size_t ns = ((size_t)kGsSmemMax - fixed) / pl.stage_bytes;
     if (ns > kGsMaxStages) ns = kGsMaxStages;
@@ -626,12 +711,16 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.act_bytes = (uint32_t)pl.act_bytes;
     prm.red_bytes = (uint32_t)pl.red_bytes;
     const bool bf16 = a_dtype == W4A16_BF16;
+    const bool bf16_math = bf16 && group != 128;   // bf16 at group 128 runs the fp16 arithmetic
     prm.km.lo = 0x000F000Fu;
-    prm.km.hi = bf16 ? 0x000F000Fu : 0x00F000F0u;
-    prm.km.magic = bf16 ? 0x43004300u : 0x64006400u;
+    prm.km.hi = bf16_math ? 0x000F000Fu : 0x00F000F0u;
+    prm.km.magic = bf16_math ? 0x43004300u : 0x64006400u;
     prm.km.m4 = 1u << 28;
     prm.km.m8 = 1u << 24;
     prm.km.m12 = 1u << 20;
+    prm.km_native = prm.km;
+    prm.km_native.hi = 0x000F000Fu;
+    prm.km_native.magic = 0x43004300u;
     if (bf16) return launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream);
     return launch_rows<__half>(prm, group, pl.smem, stream);
 }
