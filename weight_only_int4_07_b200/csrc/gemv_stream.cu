@@ -423,17 +423,33 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                         p.counters[tile] = 0;
                     }
                     named_bar(2, 32 * kGsGroupWarps);
-                    for (int c = cf + 1; c <= cl; ++c) {
-                        const float* part = p.partials + (size_t)c * M * 128;
+                    // the loads of up to kPL contributors are in flight together; the sums are
+                    // added in CTA order
+                    constexpr int kPL = NB == 1 ? 4 : 2;
+                    for (int c0 = cf + 1; c0 <= cl; c0 += kPL) {
+                        float ld[kPL][2][NB][4];
 #pragma unroll
-                        for (int rt = 0; rt < 2; ++rt)
+                        for (int j = 0; j < kPL; ++j) {
+                            const float* part = p.partials + (size_t)(c0 + j) * M * 128;
 #pragma unroll
-                            for (int b = 0; b < NB; ++b)
+                            for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                                    if (m < M) vals[rt][b][e] += __ldcg(part + m * 128 + ch);
-                                }
+                                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                                        ld[j][rt][b][e] = (m < M && c0 + j <= cl) ? __ldcg(part + m * 128 + ch) : 0.0f;
+                                    }
+                        }
+#pragma unroll
+                        for (int j = 0; j < kPL; ++j)
+#pragma unroll
+                            for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        if (c0 + j <= cl) vals[rt][b][e] += ld[j][rt][b][e];
                     }
                 }
 #pragma unroll
