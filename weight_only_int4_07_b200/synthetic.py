@@ -10,7 +10,10 @@ Distributions follow the workloads the layer is measured on:
   * weights ~ N(0, 0.02) with a fixed fraction of entries (a seeded sample without
     replacement) multiplied by a constant (outliers);
   * weights ~ 0.02 * Student-t(nu=5) in fp16;
-  * activations ~ N(0, 1) in fp16 or bf16.
+  * activations ~ N(0, 1) in fp16 or bf16;
+  * calibration inputs for the calibrated encoders: rows with correlated channels (a rank-K/8
+    common part plus independent noise) and 1% of the channels (a seeded sample) scaled by 10,
+    the outlier channels that activation-aware methods look for.
 """
 import numpy as np
 import torch
@@ -51,6 +54,20 @@ def weights_student_t(K, N, seed, nu=5.0, scale=0.02):
 
 def activations(M, K, seed, dtype=F16, std=1.0):
     return _to_bits(_rng(seed).standard_normal((M, K), dtype=np.float32) * np.float32(std), dtype)
+
+
+def calibration(S, K, seed, dtype=F16, outlier_frac=0.01, outlier_mult=10.0):
+    """S calibration rows of K input channels: Z B / sqrt(r) + 0.5 E with Z [S, r], B [r, K],
+    E [S, K] standard normal (r = max(1, K / 8)), then a seeded 1% of the channels times 10."""
+    rng = _rng(seed)
+    r = max(1, K // 8)
+    Z = rng.standard_normal((S, r), dtype=np.float32)
+    B = rng.standard_normal((r, K), dtype=np.float32)
+    x = (Z @ B) / np.float32(np.sqrt(r)) + np.float32(0.5) * rng.standard_normal((S, K), dtype=np.float32)
+    n_out = max(1, int(round(outlier_frac * K)))
+    idx = rng.choice(K, size=n_out, replace=False)
+    x[:, idx] *= np.float32(outlier_mult)
+    return _to_bits(x, dtype)
 
 
 def column_sample(N, count, seed):
