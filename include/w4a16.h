@@ -127,6 +127,43 @@ W4A16_API int w4a16_dequantize(const int32_t* codes, const void* scales, const i
                      int group, int sym, int out_dtype, void* W, void* stream);
 
 /*
+ * w4a16_gptq_workspace_bytes -- device workspace that w4a16_gptq_quantize needs for a K x N
+ * weight: 16 K^2 + 8 K N + 1024 N + 256 bytes (the damped Hessian and its factors in FP64, an FP64
+ * working copy of W, one block of propagated errors). 0 on a bad shape.
+ */
+W4A16_API size_t w4a16_gptq_workspace_bytes(int K, int N);
+
+/*
+ * w4a16_gptq_quantize -- the GPTQ calibrated encoder: the same packed output as w4a16_quantize,
+ * with every rounding error fed forward onto the input channels not yet quantized, weighted by
+ * the calibration inputs' curvature. "4.3 Weight-only INT4", section 2 "GPTQ: quantize and
+ * compensate as you go": objective ||X W - X W_hat||^2 with H = 2 X^T X (2.1); input channels
+ * fixed in order, the free ones moved by -(w_i - w_hat_i) / [H_F^-1]_ii [H_F^-1]_{:,i} (2.2),
+ * with damping, a Cholesky factorisation and block updates. Each group's RTN scale (and zero)
+ * is taken from its compensated weights when its first input channel comes up. All arithmetic
+ * is FP64; an offline, one-time step (not on the inference path).
+ * Arguments
+ *   W          device, fp16 [K, N] row-major (K input channels, N output channels).
+ *   X          device, calibration inputs [S, K] row-major, 16-bit of type x_dtype.
+ *   x_dtype    W4A16_F16 or W4A16_BF16.
+ *   S          calibration rows, >= 1.
+ *   K, N, group, sym   as for w4a16_quantize.
+ *   damp       damping as a fraction of mean(diag H), added to the diagonal (0.01 is usual);
+ *              >= 0 and finite.
+ *   codes, scales, zeros   device out, the plain layout of w4a16_quantize (zeros NULL iff sym).
+ *   workspace, ws_bytes    device, at least w4a16_gptq_workspace_bytes(K, N) bytes, 16-byte
+ *              aligned; contents on entry do not matter.
+ *   dev_status nullable device int: W4A16_ENONFINITE when W holds Inf/NaN or H + damping is not
+ *              positive definite (outputs then unspecified).
+ *   stream     cudaStream_t. About 2 K + 2 K / 128 + 4 kernel launches.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
+ * W4A16_ECUDA (host-side checks; nothing is launched on an error).
+ */
+W4A16_API int w4a16_gptq_quantize(const void* W, const void* X, int x_dtype, int S, int K, int N, int group,
+                                  int sym, double damp, int32_t* codes, void* scales, int32_t* zeros,
+                                  void* workspace, size_t ws_bytes, int* dev_status, void* stream);
+
+/*
  * w4a16_repack_bytes -- size in bytes of the tiled buffer for a K x N weight (0 on bad shape).
  */
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);

@@ -38,7 +38,7 @@ def test_headers_declare_the_entry_points():
     names = _declared_symbols()
     for required in ("w4a16_quantize", "w4a16_gemm", "w4a16_repack", "w4a16_repack_bytes",
                      "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str",
-                     "w4a16_dequantize"):
+                     "w4a16_dequantize", "w4a16_gptq_quantize", "w4a16_gptq_workspace_bytes"):
         assert required in names
 
 
@@ -166,3 +166,29 @@ def test_dequantize_rejects_bad_arguments_before_any_launch(L):
     assert call(sym=1) == native.EINVAL                   # zeros given for a symmetric weight
     assert call(zeros=None) == native.EINVAL              # asymmetric without zeros
     assert call(W=P((4 << 20) + 8)) == native.EALIGN
+
+
+def test_gptq_rejects_bad_arguments_before_any_launch(L):
+    P = ctypes.c_void_p
+    K, N = 256, 128
+    need = L.w4a16_gptq_workspace_bytes(K, N)
+    assert need == 16 * K * K + 8 * K * N + 1024 * N + 256
+    assert L.w4a16_gptq_workspace_bytes(0, N) == 0
+    ok = dict(W=P(1 << 20), X=P(2 << 20), xdt=native.F16, S=64, K=K, N=N, group=128, sym=0, damp=0.01,
+              codes=P(3 << 20), scales=P(4 << 20), zeros=P(5 << 20), ws=P(6 << 20), wsb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.w4a16_gptq_quantize(a["W"], a["X"], a["xdt"], a["S"], a["K"], a["N"], a["group"], a["sym"],
+                                     ctypes.c_double(a["damp"]), a["codes"], a["scales"], a["zeros"], a["ws"],
+                                     a["wsb"], None, None)
+    assert call(group=48) == native.EUNSUPPORTED
+    assert call(S=0) == native.EINVAL
+    assert call(xdt=5) == native.EINVAL
+    assert call(damp=-1.0) == native.EINVAL
+    assert call(damp=float("nan")) == native.EINVAL
+    assert call(zeros=None) == native.EINVAL
+    assert call(sym=1) == native.EINVAL
+    assert call(ws=None) == native.EINVAL
+    assert call(wsb=need - 1) == native.EWORKSPACE
+    assert call(X=P((2 << 20) + 2)) == native.EALIGN

@@ -14,6 +14,8 @@ from .native import (  # noqa: F401
     W4A16Error,
     w4a16_dequantize,
     w4a16_gemm,
+    w4a16_gptq_quantize,
+    w4a16_gptq_workspace_bytes,
     w4a16_quantize,
     w4a16_repack,
     w4a16_repack_bytes,

@@ -46,6 +46,11 @@ inline int launch_status() {
 int launch_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes, void* scales,
                     int32_t* zeros, int* dev_status, cudaStream_t stream);
 
+size_t gptq_workspace_bytes(int K, int N);
+int launch_gptq(const void* W, const void* X, int x_dtype, int S, int K, int N, int group, int sym, double damp,
+                int32_t* codes, void* scales, int32_t* zeros, void* workspace, int* dev_status,
+                cudaStream_t stream);
+
 int launch_dequantize(const int32_t* codes, const void* scales, const int32_t* zeros, int K, int N, int group,
                       int sym, int out_dtype, void* W, cudaStream_t stream);
 
