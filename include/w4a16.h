@@ -164,6 +164,39 @@ W4A16_API int w4a16_gptq_quantize(const void* W, const void* X, int x_dtype, int
                                   void* workspace, size_t ws_bytes, int* dev_status, void* stream);
 
 /*
+ * w4a16_awq_workspace_bytes -- device workspace of w4a16_awq_quantize for a K x N weight and S
+ * calibration rows: 8 (K^2 + K N + 2 K + 64 + P) + 256 bytes, P = ceil(S / 64) ceil(N / 64)
+ * rounded up to even. 0 on a bad shape.
+ */
+W4A16_API size_t w4a16_awq_workspace_bytes(int K, int N, int S);
+
+/*
+ * w4a16_awq_quantize -- the AWQ activation-aware encoder: input channel j of W is scaled by s_j
+ * before RTN quantization, and the layer's input must be divided by the same s_j (the caller
+ * folds 1/s into whatever produces X). "4.3 Weight-only INT4", section 3 "AWQ: find channels to
+ * protect from activations": salient channels come from the activation distribution (3.1);
+ * Y = (X S^-1)(S W), Y_hat = (X S^-1) D(Q(S W)), factors searched on calibration data and
+ * paired with clipping (3.2). Search (FP64): s_j = fp16(max(mean_s |x_sj|, 2^-14)^alpha),
+ * alpha = i / 20 for i = 0..19, scored by ||X W - (X S^-1) D(Q(S W))||^2 over the calibration
+ * rows (first minimum wins; alpha = 0 is plain RTN); then for every group and output channel
+ * the RTN range of the scaled weights shrunk by r = 1 - i / 20, i = 0..10, scored by the group's
+ * output error (first minimum wins; r = 1 is plain RTN). An offline, one-time step.
+ * Arguments
+ *   W, X, x_dtype, S, K, N, group, sym   as for w4a16_gptq_quantize.
+ *   codes, scales, zeros   device out: the plain layout of w4a16_quantize, of S W.
+ *   s_in       device out, fp16 [K]: the factors s_j (divide the layer's input by them).
+ *   workspace, ws_bytes    device, at least w4a16_awq_workspace_bytes(K, N, S) bytes, 16-byte
+ *              aligned; contents on entry do not matter.
+ *   dev_status nullable device int (reserved; nothing is reported at present).
+ *   stream     cudaStream_t. About 4 x 20 + 8 kernel launches.
+ * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
+ * W4A16_ECUDA (host-side checks; nothing is launched on an error).
+ */
+W4A16_API int w4a16_awq_quantize(const void* W, const void* X, int x_dtype, int S, int K, int N, int group,
+                                 int sym, int32_t* codes, void* scales, int32_t* zeros, void* s_in,
+                                 void* workspace, size_t ws_bytes, int* dev_status, void* stream);
+
+/*
  * w4a16_repack_bytes -- size in bytes of the tiled buffer for a K x N weight (0 on bad shape).
  */
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);

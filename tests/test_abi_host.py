@@ -38,7 +38,8 @@ def test_headers_declare_the_entry_points():
     names = _declared_symbols()
     for required in ("w4a16_quantize", "w4a16_gemm", "w4a16_repack", "w4a16_repack_bytes",
                      "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str",
-                     "w4a16_dequantize", "w4a16_gptq_quantize", "w4a16_gptq_workspace_bytes"):
+                     "w4a16_dequantize", "w4a16_gptq_quantize", "w4a16_gptq_workspace_bytes",
+                     "w4a16_awq_quantize", "w4a16_awq_workspace_bytes"):
         assert required in names
 
 
@@ -192,3 +193,26 @@ def test_gptq_rejects_bad_arguments_before_any_launch(L):
     assert call(ws=None) == native.EINVAL
     assert call(wsb=need - 1) == native.EWORKSPACE
     assert call(X=P((2 << 20) + 2)) == native.EALIGN
+
+
+def test_awq_rejects_bad_arguments_before_any_launch(L):
+    P = ctypes.c_void_p
+    K, N, S = 256, 128, 100
+    need = L.w4a16_awq_workspace_bytes(K, N, S)
+    parts = 2 * 2   # ceil(100 / 64) * ceil(128 / 64), already even
+    assert need == 8 * (K * K + K * N + 2 * K + 64 + parts) + 256
+    assert L.w4a16_awq_workspace_bytes(K, N, 0) == 0
+    ok = dict(W=P(1 << 20), X=P(2 << 20), xdt=native.F16, S=S, K=K, N=N, group=128, sym=0,
+              codes=P(3 << 20), scales=P(4 << 20), zeros=P(5 << 20), s_in=P(6 << 20), ws=P(7 << 20), wsb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.w4a16_awq_quantize(a["W"], a["X"], a["xdt"], a["S"], a["K"], a["N"], a["group"], a["sym"],
+                                    a["codes"], a["scales"], a["zeros"], a["s_in"], a["ws"], a["wsb"], None, None)
+    assert call(group=96) == native.EUNSUPPORTED
+    assert call(S=0) == native.EINVAL
+    assert call(xdt=3) == native.EINVAL
+    assert call(s_in=None) == native.EINVAL
+    assert call(zeros=None) == native.EINVAL
+    assert call(wsb=need - 8) == native.EWORKSPACE
+    assert call(s_in=P((6 << 20) + 4)) == native.EALIGN

@@ -13,6 +13,8 @@ from .native import (  # noqa: F401
     LAYOUT_TILED,
     W4A16Error,
     w4a16_dequantize,
+    w4a16_awq_quantize,
+    w4a16_awq_workspace_bytes,
     w4a16_gemm,
     w4a16_gptq_quantize,
     w4a16_gptq_workspace_bytes,

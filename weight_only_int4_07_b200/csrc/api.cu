@@ -133,6 +133,29 @@ W4A16_API int w4a16_gptq_quantize(const void* W, const void* X, int x_dtype, int
                        static_cast<cudaStream_t>(stream));
 }
 
+W4A16_API size_t w4a16_awq_workspace_bytes(int K, int N, int S) {
+    if (K <= 0 || N <= 0 || S <= 0) return 0;
+    return awq_workspace_bytes(K, N, S);
+}
+
+W4A16_API int w4a16_awq_quantize(const void* W, const void* X, int x_dtype, int S, int K, int N, int group,
+                                 int sym, int32_t* codes, void* scales, int32_t* zeros, void* s_in,
+                                 void* workspace, size_t ws_bytes, int* dev_status, void* stream) {
+    int st = check_shape(K, N, group);
+    if (st != W4A16_OK) return st;
+    if (sym != 0 && sym != 1) return W4A16_EINVAL;
+    if (x_dtype != W4A16_F16 && x_dtype != W4A16_BF16) return W4A16_EINVAL;
+    if (S < 1) return W4A16_EINVAL;
+    if (!W || !X || !codes || !scales || !s_in || !workspace) return W4A16_EINVAL;
+    if (sym ? zeros != nullptr : zeros == nullptr) return W4A16_EINVAL;
+    if (!aligned16(W) || !aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(s_in) ||
+        !aligned16(workspace) || (zeros && !aligned16(zeros)))
+        return W4A16_EALIGN;
+    if (ws_bytes < awq_workspace_bytes(K, N, S)) return W4A16_EWORKSPACE;
+    return launch_awq(W, X, x_dtype, S, K, N, group, sym, codes, scales, zeros, s_in, workspace, dev_status,
+                      static_cast<cudaStream_t>(stream));
+}
+
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym) {
     if (check_shape(K, N, group) != W4A16_OK || (sym != 0 && sym != 1)) return 0;
     if (N % kTileN != 0 || K % kTileK != 0) return 0;

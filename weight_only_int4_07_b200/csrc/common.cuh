@@ -46,7 +46,12 @@ inline int launch_status() {
 int launch_quantize(const void* W, int K, int N, int group, int sym, int32_t* codes, void* scales,
                     int32_t* zeros, int* dev_status, cudaStream_t stream);
 
+// H = 2 X^T X in FP64 for 16-bit X [S, K] (the curvature of the layer-output error).
+void launch_hessian(const void* X, int x_dtype, int S, int K, double* H, cudaStream_t stream);
 size_t gptq_workspace_bytes(int K, int N);
+size_t awq_workspace_bytes(int K, int N, int S);
+int launch_awq(const void* W, const void* X, int x_dtype, int S, int K, int N, int group, int sym, int32_t* codes,
+               void* scales, int32_t* zeros, void* s_in, void* workspace, int* dev_status, cudaStream_t stream);
 int launch_gptq(const void* W, const void* X, int x_dtype, int S, int K, int N, int group, int sym, double damp,
                 int32_t* codes, void* scales, int32_t* zeros, void* workspace, int* dev_status,
                 cudaStream_t stream);

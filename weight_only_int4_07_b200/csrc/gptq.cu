@@ -286,6 +286,15 @@ trailing_kernel(double* __restrict__ Wd, const double* __restrict__ U, const dou
 
 }  // namespace
 
+void launch_hessian(const void* X, int x_dtype, int S, int K, double* H, cudaStream_t stream) {
+    const dim3 hg((K + 31) / 32, (K + 31) / 32);
+    const uint16_t* Xb = static_cast<const uint16_t*>(X);
+    if (x_dtype == W4A16_BF16)
+        hessian_kernel<__nv_bfloat16><<<hg, dim3(32, 8), 0, stream>>>(Xb, S, K, H);
+    else
+        hessian_kernel<__half><<<hg, dim3(32, 8), 0, stream>>>(Xb, S, K, H);
+}
+
 size_t gptq_workspace_bytes(int K, int N) {
     const size_t kk = (size_t)K * K * sizeof(double);
     return 2 * kk + (size_t)K * N * sizeof(double) + (size_t)kGptqBlock * N * sizeof(double) + 256;
@@ -300,13 +309,8 @@ int launch_gptq(const void* W, const void* X, int x_dtype, int S, int K, int N, 
     double* U = H + kk;
     double* Wd = U + kk;
     double* E = Wd + (size_t)K * N;
-    const uint16_t* Xb = static_cast<const uint16_t*>(X);
 
-    const dim3 hg((K + 31) / 32, (K + 31) / 32);
-    if (x_dtype == W4A16_BF16)
-        hessian_kernel<__nv_bfloat16><<<hg, dim3(32, 8), 0, stream>>>(Xb, S, K, H);
-    else
-        hessian_kernel<__half><<<hg, dim3(32, 8), 0, stream>>>(Xb, S, K, H);
+    launch_hessian(X, x_dtype, S, K, H, stream);
     damp_kernel<<<1, 256, 0, stream>>>(H, K, damp);
     for (int j = K - 1; j >= 0; --j) {
         rchol_diag_kernel<<<1, 32, 0, stream>>>(H, K, j, dev_status);

@@ -60,6 +60,10 @@ def lib():
     L.w4a16_gptq_workspace_bytes.restype = S
     L.w4a16_gptq_quantize.argtypes = [P, P, I, I, I, I, I, I, ctypes.c_double, P, P, P, P, S, P, P]
     L.w4a16_gptq_quantize.restype = I
+    L.w4a16_awq_workspace_bytes.argtypes = [I, I, I]
+    L.w4a16_awq_workspace_bytes.restype = S
+    L.w4a16_awq_quantize.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, S, P, P]
+    L.w4a16_awq_quantize.restype = I
     L.w4a16_repack_bytes.argtypes = [I, I, I, I]
     L.w4a16_repack_bytes.restype = S
     L.w4a16_repack.argtypes = [P, P, P, I, I, I, I, P, P]
@@ -144,6 +148,36 @@ def w4a16_gptq_quantize(W, X, group, sym, damp=0.01, codes=None, scales=None, ze
                                    _ptr(dev_status), _stream())
     _check("w4a16_gptq_quantize", st)
     return codes, scales, (None if sym else zeros)
+
+
+def w4a16_awq_workspace_bytes(K, N, S) -> int:
+    return int(lib().w4a16_awq_workspace_bytes(K, N, S))
+
+
+def w4a16_awq_quantize(W, X, group, sym, codes=None, scales=None, zeros=None, s_in=None,
+                       workspace=None, dev_status=None):
+    """AWQ of fp16 W [K, N] with 16-bit calibration inputs X [S, K] on the GPU -> (codes, scales,
+    zeros, s_in): the packed S W and the fp16 factors that divide the layer's input."""
+    K, N = W.shape
+    S = X.shape[0]
+    dev = W.device
+    if codes is None:
+        codes = torch.empty((K // 8, N), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty((K // group, N), dtype=torch.float16, device=dev)
+    if zeros is None and not sym:
+        zeros = torch.empty((K // group, N // 8), dtype=torch.int32, device=dev)
+    if s_in is None:
+        s_in = torch.empty(K, dtype=torch.float16, device=dev)
+    nbytes = w4a16_awq_workspace_bytes(K, N, S)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = lib().w4a16_awq_quantize(_ptr(W), _ptr(X), _DTYPES[X.dtype], S, K, N, group, int(sym),
+                                  _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(s_in), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                  _stream())
+    _check("w4a16_awq_quantize", st)
+    return codes, scales, (None if sym else zeros), s_in
 
 
 def w4a16_dequantize(codes, scales, zeros, K, N, group, sym, dtype=None, out=None):
