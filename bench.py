@@ -498,14 +498,18 @@ def bench_naive(torch, native, synthetic, seed, steps, warmup, copies=4):
     return out
 
 
-def bench_gptq(torch, native, synthetic, seed, reps=2, S=512):
-    """The GPTQ encoder (offline, once per layer) on the four Llama-3-8B decode shapes with S
+def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv", "o")):
+    """The calibrated encoders (offline, once per layer), GPTQ and AWQ, on Llama-3-8B decode
+    shapes (by default the two with K = 4096 and N <= 6144, to keep the run short) with S
     calibration rows (fp16): device time per layer (CUDA events around the whole call), and the
-    layer-output error on the calibration inputs relative to RTN's, ||X (W - W_hat)||^2."""
+    layer-output error on the calibration inputs relative to RTN's, ||X W - X' W_hat||^2
+    (X' = X for GPTQ, X S^-1 for AWQ)."""
     dev = torch.device("cuda")
     out = {}
     stream = torch.cuda.current_stream()
     for i, (name, K, N) in enumerate(LLAMA8B_LINEARS):
+        if name not in shapes:
+            continue
         W = torch.from_numpy(synthetic.weights_normal(K, N, seed + i).view(np.int16)).view(torch.float16).to(dev)
         X = torch.from_numpy(synthetic.calibration(S, K, seed + 50 + i).view(np.int16)).view(torch.float16).to(dev)
         ws = torch.empty(native.w4a16_gptq_workspace_bytes(K, N), dtype=torch.uint8, device=dev)
@@ -526,9 +530,25 @@ def bench_gptq(torch, native, synthetic, seed, reps=2, S=512):
             What = native.w4a16_dequantize(qq[0], qq[1], qq[2], K, N, GROUP, SYM).double()
             return float(((X64 @ (W64 - What)) ** 2).sum())
 
-        out[name] = {"K": K, "N": N, "calib_rows": S, "ms": statistics.mean(ms),
-                     "output_error_vs_rtn": err(q) / err(r)}
-        del W, X, ws, q, r, X64, W64
+        # AWQ on the same layer: the encoded S W with inputs divided by s
+        wsa = torch.empty(native.w4a16_awq_workspace_bytes(K, N, S), dtype=torch.uint8, device=dev)
+        a = native.w4a16_awq_quantize(W, X, GROUP, SYM, workspace=wsa)   # warm-up
+        torch.cuda.synchronize()
+        ms_awq = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            a = native.w4a16_awq_quantize(W, X, GROUP, SYM, workspace=wsa)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_awq.append(e0.elapsed_time(e1))
+        Da = native.w4a16_dequantize(a[0], a[1], a[2], K, N, GROUP, SYM).double()
+        e_awq = float(((X64 @ W64 - (X64 / a[3].double()) @ Da) ** 2).sum())
+        e_rtn = err(r)
+        out[name] = {"K": K, "N": N, "calib_rows": S, "gptq_ms": statistics.mean(ms),
+                     "gptq_output_error_vs_rtn": err(q) / e_rtn, "awq_ms": statistics.mean(ms_awq),
+                     "awq_output_error_vs_rtn": e_awq / e_rtn}
+        del W, X, ws, wsa, q, r, a, Da, X64, W64
         torch.cuda.empty_cache()
     return out
 
@@ -743,10 +763,10 @@ def run_ours(args):
             r["fused_us"] = fused_us
             r["fused_speedup"] = None if fused_us is None else r["total_us"] / fused_us
 
-    # the GPTQ encoder (offline), per 8B layer shape
-    gptq = None
-    if not args.skip_gptq:
-        gptq = bench_gptq(torch, native, synthetic, replica_seed(9500, rank))
+    # the calibrated encoders (offline), per 8B layer shape
+    encoders = None
+    if not args.skip_encoders:
+        encoders = bench_encoders(torch, native, synthetic, replica_seed(9500, rank))
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -772,7 +792,7 @@ def run_ours(args):
                            "timing": "CUDA graph replay of one step, CUDA events"},
                 "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
                 "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
-                "m1_70b": m1_70b, "m256": m256, "naive": naive, "gptq": gptq}
+                "m1_70b": m1_70b, "m256": m256, "naive": naive, "encoders": encoders}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -820,7 +840,7 @@ def main(argv=None):
     ap.add_argument("--skip-70b", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-naive", action="store_true")
-    ap.add_argument("--skip-gptq", action="store_true")
+    ap.add_argument("--skip-encoders", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--single", default=None, help="K,N,M: a few launches of one GEMM, untimed")
     ap.add_argument("--dtype", choices=("f16", "bf16"), default="f16")
