@@ -553,6 +553,65 @@ def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv",
     return out
 
 
+def bench_crossover(torch, native, synthetic, seed, Ms=(1, 16, 64, 128, 256, 512, 1024, 2048), reps=6):
+    """W4A16 against the W8A8 FP8 path on the (8192, 28672) sweep layer, bf16 activations, per
+    batch size M: device time of one W4A16 GEMM (the library's dispatch on the tiled layout) and of
+    one FP8 step (per-row activation quantization + the kind::f8f6f4 GEMM), each on two rotating
+    weight copies (244 MB and 470 MB), and the smallest M where the FP8 step is faster -- the
+    crossover of the pages' roofline argument."""
+    dev = torch.device("cuda")
+    K, N = SWEEP_K, SWEEP_N
+    W = torch.from_numpy(synthetic.weights_outliers(K, N, seed).view(np.int16)).view(torch.float16).to(dev)
+    codes, scales, zeros = native.w4a16_quantize(W, GROUP, SYM)
+    tiled = [native.w4a16_repack(codes, scales, zeros, K, N, GROUP, SYM) for _ in range(2)]
+    f8 = [native.w4a16_fp8_quantize_weights(W) for _ in range(2)]
+    del W, codes, scales, zeros
+    stream = torch.cuda.current_stream()
+    out = []
+    for M in Ms:
+        A = torch.from_numpy(synthetic.activations(M, K, seed + M, dtype=synthetic.BF16).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(native.w4a16_workspace_bytes(M, N, K, GROUP), 16), dtype=torch.uint8, device=dev)
+        Aq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        sa = torch.empty(M, dtype=torch.float32, device=dev)
+
+        def w4(i):
+            native.w4a16_gemm(A, tiled[i % 2], None, None, N, GROUP, SYM, layout=native.LAYOUT_TILED, C=C,
+                              workspace=ws)
+
+        def w8(i, quant=True):
+            if quant:
+                native.w4a16_fp8_quantize_acts(A, Aq, sa)
+            native.w4a16_fp8_gemm(Aq, sa, f8[i % 2][0], f8[i % 2][1], C=C)
+
+        res = {}
+        for name, fn in (("w4a16", w4), ("fp8_step", w8), ("fp8_gemm", lambda i: w8(i, quant=False))):
+            for i in range(3):
+                fn(i)
+            torch.cuda.synchronize()
+            torch.cuda._sleep(int(20e6))
+            evs = []
+            for i in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn(i)
+                e1.record(stream)
+                evs.append((e0, e1))
+            torch.cuda.synchronize()
+            res[name] = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+        flops = gemm_flops(M, K, N)
+        out.append({"M": M, "w4a16_us": res["w4a16"], "fp8_step_us": res["fp8_step"],
+                    "fp8_gemm_us": res["fp8_gemm"], "w4a16_tflops": flops / (res["w4a16"] * 1e-6) / 1e12,
+                    "fp8_step_tflops": flops / (res["fp8_step"] * 1e-6) / 1e12})
+        del A, C, ws, Aq, sa
+    faster = [r["M"] for r in out if r["fp8_step_us"] < r["w4a16_us"]]
+    del tiled, f8
+    torch.cuda.empty_cache()
+    return {"layer": {"K": K, "N": N, "acts": "bf16"}, "points": out,
+            "crossover_M": (min(faster) if faster else None)}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def host_cores():
     try:
@@ -768,6 +827,11 @@ def run_ours(args):
     if not args.skip_encoders:
         encoders = bench_encoders(torch, native, synthetic, replica_seed(9500, rank))
 
+    # W4A16 against the W8A8 FP8 path across batch sizes (the crossover)
+    crossover = None
+    if not args.skip_crossover:
+        crossover = bench_crossover(torch, native, synthetic, replica_seed(9700, rank))
+
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         threads = host_cores()
@@ -792,7 +856,8 @@ def run_ours(args):
                            "timing": "CUDA graph replay of one step, CUDA events"},
                 "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
                 "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
-                "m1_70b": m1_70b, "m256": m256, "naive": naive, "encoders": encoders}
+                "m1_70b": m1_70b, "m256": m256, "naive": naive, "encoders": encoders,
+                "crossover": crossover}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -841,6 +906,7 @@ def main(argv=None):
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-naive", action="store_true")
     ap.add_argument("--skip-encoders", action="store_true")
+    ap.add_argument("--skip-crossover", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--single", default=None, help="K,N,M: a few launches of one GEMM, untimed")
     ap.add_argument("--dtype", choices=("f16", "bf16"), default="f16")

@@ -197,6 +197,32 @@ W4A16_API int w4a16_awq_quantize(const void* W, const void* X, int x_dtype, int 
                                  void* workspace, size_t ws_bytes, int* dev_status, void* stream);
 
 /*
+ * The W8A8 comparison path (FP8 E4M3 weights and activations, tcgen05 kind::f8f6f4 GEMM) that
+ * W4A16 is measured against: "INT8 vs INT4 Quantization, in depth", section "Two regimes: waiting
+ * for memory, waiting for math" (8-bit weights double the bytes read but the 8-bit tensor rate
+ * doubles the math rate; the crossover batch follows from the roofline). Not a W4A16 format.
+ * Codes: E4M3 round-to-nearest-even of x / s (computed in FP64), saturated to +-448; scales
+ * s = fp32(amax / 448) (1 when amax = 0), per output channel (weights) and per row (activations).
+ *
+ * w4a16_fp8_quantize_weights -- W fp16 [K, N] (device) -> Wq uint8 [N, K] (device, one row of K
+ *   codes per output channel) and w_scales fp32 [N] (device). K % 128 == 0 and N % 128 == 0
+ *   (else W4A16_EUNSUPPORTED). An offline step.
+ * w4a16_fp8_quantize_acts -- A [M, K] of a_dtype (device) -> Aq uint8 [M, K] and a_scales fp32 [M]
+ *   (device). K % 128 == 0. Part of every W8A8 step (activations change each step).
+ * w4a16_fp8_gemm -- C[m, n] = (sum_k Aq[m, k] Wq[n, k]) a_scales[m] w_scales[n], FP32
+ *   accumulation, C [M, N] of c_dtype (device). M >= 1; K % 128 == 0; N % 128 == 0.
+ *   dev_status (nullable) receives W4A16_ETIMEOUT if a bounded pipeline wait expired.
+ * All three: every pointer 16-byte aligned (W4A16_EALIGN), the caller owns every buffer, no
+ * allocation or synchronisation; W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED or
+ * W4A16_ECUDA.
+ */
+W4A16_API int w4a16_fp8_quantize_weights(const void* W, int K, int N, uint8_t* Wq, float* w_scales, void* stream);
+W4A16_API int w4a16_fp8_quantize_acts(const void* A, int a_dtype, int M, int K, uint8_t* Aq, float* a_scales,
+                                      void* stream);
+W4A16_API int w4a16_fp8_gemm(const uint8_t* Aq, const float* a_scales, int M, int K, const uint8_t* Wq,
+                             const float* w_scales, int N, void* C, int c_dtype, int* dev_status, void* stream);
+
+/*
  * w4a16_repack_bytes -- size in bytes of the tiled buffer for a K x N weight (0 on bad shape).
  */
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);

@@ -39,7 +39,8 @@ def test_headers_declare_the_entry_points():
     for required in ("w4a16_quantize", "w4a16_gemm", "w4a16_repack", "w4a16_repack_bytes",
                      "w4a16_workspace_bytes", "w4a16_select_kernel", "w4a16_status_str",
                      "w4a16_dequantize", "w4a16_gptq_quantize", "w4a16_gptq_workspace_bytes",
-                     "w4a16_awq_quantize", "w4a16_awq_workspace_bytes"):
+                     "w4a16_awq_quantize", "w4a16_awq_workspace_bytes",
+                     "w4a16_fp8_quantize_weights", "w4a16_fp8_quantize_acts", "w4a16_fp8_gemm"):
         assert required in names
 
 
@@ -216,3 +217,19 @@ def test_awq_rejects_bad_arguments_before_any_launch(L):
     assert call(zeros=None) == native.EINVAL
     assert call(wsb=need - 8) == native.EWORKSPACE
     assert call(s_in=P((6 << 20) + 4)) == native.EALIGN
+
+
+def test_fp8_rejects_bad_arguments_before_any_launch(L):
+    P = ctypes.c_void_p
+    a, b, c = P(1 << 20), P(2 << 20), P(3 << 20)
+    assert L.w4a16_fp8_quantize_weights(a, 200, 128, b, c, None) == native.EUNSUPPORTED
+    assert L.w4a16_fp8_quantize_weights(a, 256, 128, None, c, None) == native.EINVAL
+    assert L.w4a16_fp8_quantize_weights(P((1 << 20) + 2), 256, 128, b, c, None) == native.EALIGN
+    assert L.w4a16_fp8_quantize_acts(a, 0, 0, 256, b, c, None) == native.EINVAL
+    assert L.w4a16_fp8_quantize_acts(a, 4, 1, 256, b, c, None) == native.EINVAL
+    assert L.w4a16_fp8_quantize_acts(a, 0, 1, 100, b, c, None) == native.EUNSUPPORTED
+    d = P(4 << 20)
+    assert L.w4a16_fp8_gemm(a, b, 1, 256, c, d, 100, P(5 << 20), 0, None, None) == native.EUNSUPPORTED
+    assert L.w4a16_fp8_gemm(a, b, 0, 256, c, d, 128, P(5 << 20), 0, None, None) == native.EINVAL
+    assert L.w4a16_fp8_gemm(a, b, 1, 256, c, d, 128, P(5 << 20), 2, None, None) == native.EINVAL
+    assert L.w4a16_fp8_gemm(a, b, 1, 256, c, P((4 << 20) + 4), 128, P(5 << 20), 0, None, None) == native.EALIGN

@@ -15,6 +15,9 @@ from .native import (  # noqa: F401
     w4a16_dequantize,
     w4a16_awq_quantize,
     w4a16_awq_workspace_bytes,
+    w4a16_fp8_gemm,
+    w4a16_fp8_quantize_acts,
+    w4a16_fp8_quantize_weights,
     w4a16_gemm,
     w4a16_gptq_quantize,
     w4a16_gptq_workspace_bytes,

@@ -156,6 +156,35 @@ W4A16_API int w4a16_awq_quantize(const void* W, const void* X, int x_dtype, int 
                       static_cast<cudaStream_t>(stream));
 }
 
+W4A16_API int w4a16_fp8_quantize_weights(const void* W, int K, int N, uint8_t* Wq, float* w_scales, void* stream) {
+    if (K <= 0 || N <= 0 || K % 128 != 0 || N % 128 != 0) return K > 0 && N > 0 ? W4A16_EUNSUPPORTED : W4A16_EINVAL;
+    if (!W || !Wq || !w_scales) return W4A16_EINVAL;
+    if (!aligned16(W) || !aligned16(Wq) || !aligned16(w_scales)) return W4A16_EALIGN;
+    return launch_fp8_quantize_weights(W, K, N, Wq, w_scales, static_cast<cudaStream_t>(stream));
+}
+
+W4A16_API int w4a16_fp8_quantize_acts(const void* A, int a_dtype, int M, int K, uint8_t* Aq, float* a_scales,
+                                      void* stream) {
+    if (M < 1 || K <= 0) return W4A16_EINVAL;
+    if (K % 128 != 0) return W4A16_EUNSUPPORTED;
+    if (a_dtype != W4A16_F16 && a_dtype != W4A16_BF16) return W4A16_EINVAL;
+    if (!A || !Aq || !a_scales) return W4A16_EINVAL;
+    if (!aligned16(A) || !aligned16(Aq) || !aligned16(a_scales)) return W4A16_EALIGN;
+    return launch_fp8_quantize_acts(A, a_dtype, M, K, Aq, a_scales, static_cast<cudaStream_t>(stream));
+}
+
+W4A16_API int w4a16_fp8_gemm(const uint8_t* Aq, const float* a_scales, int M, int K, const uint8_t* Wq,
+                             const float* w_scales, int N, void* C, int c_dtype, int* dev_status, void* stream) {
+    if (M < 1 || K <= 0 || N <= 0) return W4A16_EINVAL;
+    if (K % 128 != 0 || N % 128 != 0) return W4A16_EUNSUPPORTED;
+    if (c_dtype != W4A16_F16 && c_dtype != W4A16_BF16) return W4A16_EINVAL;
+    if (!Aq || !a_scales || !Wq || !w_scales || !C) return W4A16_EINVAL;
+    if (!aligned16(Aq) || !aligned16(Wq) || !aligned16(C) || !aligned16(a_scales) || !aligned16(w_scales))
+        return W4A16_EALIGN;
+    return launch_fp8_gemm(Aq, a_scales, M, K, Wq, w_scales, N, C, c_dtype, dev_status,
+                           static_cast<cudaStream_t>(stream));
+}
+
 W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym) {
     if (check_shape(K, N, group) != W4A16_OK || (sym != 0 && sym != 1)) return 0;
     if (N % kTileN != 0 || K % kTileK != 0) return 0;

@@ -50,6 +50,10 @@ int launch_quantize(const void* W, int K, int N, int group, int sym, int32_t* co
 void launch_hessian(const void* X, int x_dtype, int S, int K, double* H, cudaStream_t stream);
 size_t gptq_workspace_bytes(int K, int N);
 size_t awq_workspace_bytes(int K, int N, int S);
+int launch_fp8_quantize_weights(const void* W, int K, int N, uint8_t* Wq, float* sw, cudaStream_t stream);
+int launch_fp8_quantize_acts(const void* A, int a_dtype, int M, int K, uint8_t* Aq, float* sa, cudaStream_t stream);
+int launch_fp8_gemm(const uint8_t* Aq, const float* sa, int M, int K, const uint8_t* Wq, const float* sw, int N,
+                    void* C, int c_dtype, int* dev_status, cudaStream_t stream);
 int launch_awq(const void* W, const void* X, int x_dtype, int S, int K, int N, int group, int sym, int32_t* codes,
                void* scales, int32_t* zeros, void* s_in, void* workspace, int* dev_status, cudaStream_t stream);
 int launch_gptq(const void* W, const void* X, int x_dtype, int S, int K, int N, int group, int sym, double damp,

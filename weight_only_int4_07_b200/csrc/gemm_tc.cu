@@ -301,6 +301,21 @@ bool make_act_map(CUtensorMap* map, const void* A, int M, int K, int box_rows, b
     return r == CUDA_SUCCESS;
 }
 
+// An 8-bit matrix [rows, K] (row-major, K bytes per row) as a 2-D tensor map: box 128 (K) x
+// box_rows, 128-byte swizzle; rows past the end read as zero.
+bool make_u8_map(CUtensorMap* map, const void* base, int rows, int K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <int BN, typename T>

@@ -189,6 +189,25 @@ __device__ __forceinline__ void mma4_f16_ss_commit(uint32_t d_tmem, uint64_t a_d
         : "memory");
 }
 
+// The same for kind::f8f6f4 (8-bit operands): four MMAs of K = 32 bytes each, so one 128-byte
+// swizzled row of K. The instruction descriptor has the same fields; E4M3 is format code 0 for
+// A and B.
+__device__ __forceinline__ void mma4_f8_ss_commit(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate, uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %3, 0;\n\t"
+        "setp.eq.b32 t, %2, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %5, %2, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %6, %7, %2, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %8, %9, %2, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %10, %11, %2, t;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%1];\n\t}" ::"r"(d_tmem),
+        "r"(smem_u32(bar)), "r"(idesc), "r"(accumulate), "l"(a_desc), "l"(b_desc), "l"(a_desc + 2), "l"(b_desc + 2),
+        "l"(a_desc + 4), "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
+        : "memory");
+}
+
 // The mbarrier arrives once every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -64,6 +64,12 @@ def lib():
     L.w4a16_awq_workspace_bytes.restype = S
     L.w4a16_awq_quantize.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, S, P, P]
     L.w4a16_awq_quantize.restype = I
+    L.w4a16_fp8_quantize_weights.argtypes = [P, I, I, P, P, P]
+    L.w4a16_fp8_quantize_weights.restype = I
+    L.w4a16_fp8_quantize_acts.argtypes = [P, I, I, I, P, P, P]
+    L.w4a16_fp8_quantize_acts.restype = I
+    L.w4a16_fp8_gemm.argtypes = [P, P, I, I, P, P, I, P, I, P, P]
+    L.w4a16_fp8_gemm.restype = I
     L.w4a16_repack_bytes.argtypes = [I, I, I, I]
     L.w4a16_repack_bytes.restype = S
     L.w4a16_repack.argtypes = [P, P, P, I, I, I, I, P, P]
@@ -178,6 +184,39 @@ def w4a16_awq_quantize(W, X, group, sym, codes=None, scales=None, zeros=None, s_
                                   _stream())
     _check("w4a16_awq_quantize", st)
     return codes, scales, (None if sym else zeros), s_in
+
+
+def w4a16_fp8_quantize_weights(W):
+    """fp16 W [K, N] -> (Wq uint8 [N, K] E4M3 codes, w_scales float32 [N]) on the GPU."""
+    K, N = W.shape
+    Wq = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    sw = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check("w4a16_fp8_quantize_weights",
+           lib().w4a16_fp8_quantize_weights(_ptr(W), K, N, _ptr(Wq), _ptr(sw), _stream()))
+    return Wq, sw
+
+
+def w4a16_fp8_quantize_acts(A, Aq=None, sa=None):
+    """16-bit A [M, K] -> (Aq uint8 [M, K] E4M3 codes, a_scales float32 [M]) on the GPU."""
+    M, K = A.shape
+    if Aq is None:
+        Aq = torch.empty((M, K), dtype=torch.uint8, device=A.device)
+    if sa is None:
+        sa = torch.empty(M, dtype=torch.float32, device=A.device)
+    _check("w4a16_fp8_quantize_acts",
+           lib().w4a16_fp8_quantize_acts(_ptr(A), _DTYPES[A.dtype], M, K, _ptr(Aq), _ptr(sa), _stream()))
+    return Aq, sa
+
+
+def w4a16_fp8_gemm(Aq, sa, Wq, sw, dtype=None, C=None, dev_status=None):
+    """C[M, N] = (Aq . Wq^T) * sa[m] * sw[n], FP32 accumulation, C in `dtype` (fp16 default)."""
+    M, K = Aq.shape
+    N = Wq.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float16 if dtype is None else dtype, device=Aq.device)
+    _check("w4a16_fp8_gemm", lib().w4a16_fp8_gemm(_ptr(Aq), _ptr(sa), M, K, _ptr(Wq), _ptr(sw), N, _ptr(C),
+                                                  _DTYPES[C.dtype], _ptr(dev_status), _stream()))
+    return C
 
 
 def w4a16_dequantize(codes, scales, zeros, K, N, group, sym, dtype=None, out=None):
