@@ -553,7 +553,7 @@ def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv",
     return out
 
 
-def bench_crossover(torch, native, synthetic, seed, Ms=(1, 16, 64, 128, 256, 512, 1024, 2048), reps=6):
+def bench_crossover(torch, native, synthetic, seed, Ms=(1, 4, 8, 16, 64, 128, 256, 512, 1024, 2048), reps=6):
     """W4A16 against the W8A8 FP8 path on the (8192, 28672) sweep layer, bf16 activations, per
     batch size M: device time of one W4A16 GEMM (the library's dispatch on the tiled layout) and of
     one FP8 step (per-row activation quantization + the kind::f8f6f4 GEMM), each on two rotating

@@ -81,12 +81,15 @@ def test_repack_bytes(L):
 
 
 def test_select_kernel_and_workspace_are_host_only(L):
-    for M in (1, 2, 16, 17, 32, 256, 2048):
+    for M in (1, 2, 8, 16, 17, 32, 256, 2048):
         k = native.w4a16_select_kernel(M, 4096, 4096, 128)
         assert k in (native.KERNEL_GEMV, native.KERNEL_TC)
-        # decode-sized M streams the weights (the decode GEMV); larger M uses the tensor-core GEMM
-        assert k == (native.KERNEL_GEMV if M <= 16 else native.KERNEL_TC)
+        # up to 8 rows the decode GEMV (whole K or K slices); 16 rows at K = 4096 need K slices,
+        # where the two-tile decode kernel loses to the tensor-core GEMM; larger M: tensor cores
+        assert k == (native.KERNEL_GEMV if M <= 8 else native.KERNEL_TC)
         assert native.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
+    # 12 rows at K = 1024 fit in shared memory whole: the decode GEMV
+    assert native.w4a16_select_kernel(12, 4096, 1024, 128) == native.KERNEL_GEMV
     assert native.w4a16_workspace_bytes(0, 4096, 4096, 128) == 0
     assert native.w4a16_workspace_bytes(1, 4096, 4000, 128) == 0
 

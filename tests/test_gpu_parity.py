@@ -520,8 +520,9 @@ def test_gemm_stream_llama70b_decode_sampled(K, N):
 
 @pytest.mark.parametrize("M", [6, 8, 9, 16])
 def test_gemm_auto_sweep_shape_sampled_skinny(M):
-    """M rows of A too long for the decode kernel's shared memory: the AUTO dispatch takes the
-    tensor-core GEMM, still within the bound."""
+    """M rows of A too long to sit in the decode kernel's shared memory whole: the AUTO dispatch
+    runs the decode kernel over K slices (one launch each, FP32 outputs added in slice order),
+    still within the bound."""
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9900 + M, a_dtype)
@@ -529,6 +530,31 @@ def test_gemm_auto_sweep_shape_sampled_skinny(M):
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", [
+    (16, 8192, 9600, 128, 0, 1),    # eight K slices of 1024: 8-unit tiles, 4 or 5 units per CTA
+    (8, 8192, 6144, 32, 1, 0),      # two slices (the smaller g32 sym records leave room)
+    (12, 16384, 8192, 64, 0, 1),    # eight slices of 2048
+])
+def test_gemm_stream_k_slices_full_output(M, K, N, group, sym, a_dtype):
+    """The decode kernel over K slices: full output within the bound, stages that run across a
+    tile boundary of the slice (two copies), counters left at zero, and a second call identical."""
+    kind = "student_t" if sym else "outliers"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 170 + M)
+    Ab, A = _acts(M, K, 1700 + M, a_dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_GEMV, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+    assert torch.count_nonzero(ws[:65536]).item() == 0
+    C2 = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                           kernel=native.KERNEL_GEMV, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(C.view(torch.int16), C2.view(torch.int16))
 
 
 # ----------------------------------------------------------------------------- naive path

@@ -54,13 +54,19 @@ const char* kernel_name(int k) {
     }
 }
 
-// The dispatch proper (tiled layout), without the environment override. Up to M = 16 the layer is
-// bound by the weight stream and the stream-K decode GEMV serves it; above, the tensor-core GEMM.
+// The dispatch proper (tiled layout), without the environment override. For small M the layer is
+// bound by the weight stream and the stream-K decode GEMV serves it (over K slices when the M rows
+// of A do not fit in its shared memory at once); above, the tensor-core GEMM. Measured on the (8192, 28672), (28672, 8192) and (4096, 28672) layers (bf16, g128): the decode
+// kernel beats the tensor-core GEMM by 2-3x for M <= 8 whether K is held whole or in slices; for
+// M = 9..16 (two 8-row MMA tiles) it wins only when K is held whole, and is up to 1.8x slower when
+// K needs 8 or more slices.
 int dispatch(int M, int N, int K, int group) {
-    (void)N;
-    (void)K;
-    (void)group;
-    return M <= 16 ? W4A16_KERNEL_GEMV : W4A16_KERNEL_TC;
+    if (M > 16) return W4A16_KERNEL_TC;
+    if (M <= 8) return W4A16_KERNEL_GEMV;
+    int n_sm = gemv_stream_sm_count();
+    if (n_sm <= 0) n_sm = 148;
+    const GemvStreamPlan q = plan_gemv_stream(M, N, K, group, 0, n_sm);
+    return q.ok && q.slices == 1 ? W4A16_KERNEL_GEMV : W4A16_KERNEL_TC;
 }
 
 }  // namespace

@@ -92,7 +92,8 @@ struct GemvStreamPlan {
     int ns;               // pipeline stages
     int ctas;             // persistent CTAs (one per SM)
     size_t row_bytes, act_bytes, red_bytes, stage_bytes, smem;
-    size_t partial_bytes; // workspace after the counters
+    size_t partial_bytes; // workspace after the counters (cut-tile sums, then the slices' outputs)
+    int slices;           // launches over equal K slices (1: the whole K at once)
 };
 GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm);
 int gemv_stream_sm_count();

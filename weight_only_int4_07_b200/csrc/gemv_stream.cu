@@ -190,6 +190,11 @@ struct GsParams {
     uint32_t stage_bytes, row_bytes, act_bytes, red_bytes;
     GsMasks km;
     GsMasks km_native;   // bf16 masks, for bf16 rows kept in bf16 at group 128
+    // K slice of this launch: A points at its first column, rows lda elements apart; the slice's
+    // units are K-steps c0 .. c0 + K/128 of every tile of a K_total/128 = ktot-step weight; with
+    // out_f32 set the FP32 sums go there ([M][N]) instead of C
+    int lda, c0, ktot;
+    float* out_f32;
 };
 
 // NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
@@ -251,8 +256,20 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                                                                         : kGsUnitsPerStage;
         const uint32_t bytes = (uint32_t)n * R;
         mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(stages + (size_t)s * stage_bytes, p.tiled + (size_t)(u0 + (long long)st * kGsUnitsPerStage) * R,
-                 bytes, &full[s]);
+        const long long ua = u0 + (long long)st * kGsUnitsPerStage;
+        uint8_t* dst = stages + (size_t)s * stage_bytes;
+        if (p.ktot == steps) {
+            bulk_g2s(dst, p.tiled + (size_t)ua * R, bytes, &full[s]);
+        } else {
+            // a K slice: units of one tile are contiguous; a stage may run into the next tile
+            const long long t = ua / steps;
+            const int cc = (int)(ua - t * steps);
+            const int n1 = steps - cc < n ? steps - cc : n;
+            bulk_g2s(dst, p.tiled + ((size_t)t * p.ktot + p.c0 + cc) * R, (uint32_t)n1 * R, &full[s]);
+            if (n1 < n)
+                bulk_g2s(dst + (size_t)n1 * R, p.tiled + ((size_t)(t + 1) * p.ktot + p.c0) * R, (uint32_t)(n - n1) * R,
+                         &full[s]);
+        }
         atomicAdd(&issued[s], 1);
     };
     if (threadIdx.x == 0)
@@ -283,7 +300,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (c0 + j * kGsThreads < vpr)
-                        vv[j] = *reinterpret_cast<const uint4*>(A + (size_t)m * K +
+                        vv[j] = *reinterpret_cast<const uint4*>(A + (size_t)m * p.lda +
                                                                  8 * ((c0 + j * kGsThreads + cta * 64) % vpr));
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
@@ -463,7 +480,10 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                                 float y = vals[rt][b][e];
                                 if constexpr (kConv)   // undo the row's 2^-k
                                     if (!wide) y *= __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
-                                C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(y);
+                                if (p.out_f32)
+                                    p.out_f32[(size_t)m * N + n0 + ch] = y;
+                                else
+                                    C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(y);
                             }
                         }
             } else {
@@ -658,6 +678,17 @@ int launch_rows(const GsParams& prm, int group, size_t smem, cudaStream_t stream
     return launch_group<1, T, false>(prm, group, smem, stream);
 }
 
+// C = sum over the S slices of the FP32 partial outputs, in slice order.
+template <typename T>
+__global__ void __launch_bounds__(256) gs_slice_reduce_kernel(const float* __restrict__ parts, int S, size_t MN,
+                                                              T* __restrict__ C) {
+    for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < MN; i += (size_t)gridDim.x * 256) {
+        float y = 0.0f;
+        for (int k = 0; k < S; ++k) y += parts[(size_t)k * MN + i];
+        C[i] = Act<T>::from_f32(y);
+    }
+}
+
 int sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -672,13 +703,13 @@ int sm_count() {
 
 }  // namespace
 
-GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm) {
+namespace {
+
+// The layout of one launch over a K slice of Ks input channels.
+GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
     GemvStreamPlan pl = {};
-    if (M < 1 || M > 16 || K % 128 != 0 || N % 128 != 0 || K < 128 || N < 128) return pl;
-    if (group != 32 && group != 64 && group != 128) return pl;
-    if (N / 128 > kGemvStreamMaxTiles) return pl;
-    const TiledLayout L = tiled_layout(K, N, group, sym);
-    const size_t units = (size_t)(K / 128);
+    const TiledLayout L = tiled_layout(Ks, N, group, sym);   // the record size does not depend on K
+    const size_t units = (size_t)(Ks / 128);
     pl.row_bytes = 320 * units + ((units & 1) ? 0 : 64);          // 80-byte blocks; rows 64 mod 128 apart
     pl.act_bytes = ((size_t)M * pl.row_bytes + 127) & ~(size_t)127;
     pl.red_bytes = (size_t)2 * 3 * M * 128 * 4;
@@ -691,11 +722,32 @@ GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_s
     if (ns < kGsMinStages) return pl;
     pl.ns = (int)ns;
     pl.smem = fixed + ns * pl.stage_bytes;
-    const long long total_units = (long long)(N / 128) * (K / 128);
+    const long long total_units = (long long)(N / 128) * (Ks / 128);
     pl.ctas = n_sm > 0 ? (int)(total_units < n_sm ? total_units : n_sm) : 0;
-    pl.partial_bytes = (size_t)(n_sm > 0 ? n_sm : 0) * M * 128 * 4;
     pl.ok = pl.ctas > 0;
     return pl;
+}
+
+}  // namespace
+
+// The whole K in one launch when the M rows of A fit in shared memory beside three stages;
+// otherwise K is cut into S equal slices (S a power of two dividing K / 128), one launch each,
+// whose FP32 outputs a last kernel adds in slice order.
+GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm) {
+    GemvStreamPlan pl = {};
+    if (M < 1 || M > 16 || K % 128 != 0 || N % 128 != 0 || K < 128 || N < 128) return pl;
+    if (group != 32 && group != 64 && group != 128) return pl;
+    if (N / 128 > kGemvStreamMaxTiles) return pl;
+    for (int S = 1; S <= 64 && (K / 128) % S == 0; S *= 2) {
+        pl = plan_slice(M, N, K / S, group, sym, n_sm);
+        if (pl.ok) {
+            pl.slices = S;
+            pl.partial_bytes = (size_t)2 * (n_sm > 0 ? n_sm : 0) * M * 128 * 4 +
+                               (S > 1 ? (size_t)S * M * N * 4 : 0);
+            return pl;
+        }
+    }
+    return GemvStreamPlan{};
 }
 
 int gemv_stream_sm_count() { return sm_count(); }
@@ -705,16 +757,18 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     const GemvStreamPlan pl = plan_gemv_stream(M, N, K, group, sym, sm_count());
     if (!pl.ok) return W4A16_EUNSUPPORTED;
     if (!workspace) return W4A16_EWORKSPACE;
+    const int S = pl.slices;
+    const int Ks = K / S;
     const TiledLayout L = tiled_layout(K, N, group, sym);
     GsParams prm = {};
-    prm.A = A;
     prm.tiled = static_cast<const uint8_t*>(tiled);
     prm.C = C;
     prm.counters = static_cast<int*>(workspace);
     prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kGemvStreamCounterBytes);
+    float* slice_out = prm.partials + (size_t)2 * sm_count() * M * 128;
     prm.dev_status = dev_status;
     prm.M = M;
-    prm.K = K;
+    prm.K = Ks;
     prm.N = N;
     prm.sym = sym;
     prm.ns = pl.ns;
@@ -726,6 +780,8 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.row_bytes = (uint32_t)pl.row_bytes;
     prm.act_bytes = (uint32_t)pl.act_bytes;
     prm.red_bytes = (uint32_t)pl.red_bytes;
+    prm.lda = K;
+    prm.ktot = K / 128;
     const bool bf16 = a_dtype == W4A16_BF16;
     const bool bf16_math = bf16 && group != 128;   // bf16 at group 128 runs the fp16 arithmetic
     prm.km.lo = 0x000F000Fu;
@@ -737,8 +793,25 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.km_native = prm.km;
     prm.km_native.hi = 0x000F000Fu;
     prm.km_native.magic = 0x43004300u;
-    if (bf16) return launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream);
-    return launch_rows<__half>(prm, group, pl.smem, stream);
+    for (int sl = 0; sl < S; ++sl) {
+        prm.A = static_cast<const uint16_t*>(A) + (size_t)sl * Ks;
+        prm.c0 = sl * (Ks / 128);
+        prm.out_f32 = S > 1 ? slice_out + (size_t)sl * M * N : nullptr;
+        const int st = bf16 ? launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream)
+                            : launch_rows<__half>(prm, group, pl.smem, stream);
+        if (st != W4A16_OK) return st;
+    }
+    if (S > 1) {
+        const size_t MN = (size_t)M * N;
+        const unsigned blocks = (unsigned)((MN + 255) / 256 < 2048 ? (MN + 255) / 256 : 2048);
+        if (bf16)
+            gs_slice_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(slice_out, S, MN,
+                                                                              static_cast<__nv_bfloat16*>(C));
+        else
+            gs_slice_reduce_kernel<__half><<<blocks, 256, 0, stream>>>(slice_out, S, MN, static_cast<__half*>(C));
+        return launch_status();
+    }
+    return W4A16_OK;
 }
 
 }  // namespace w4a16
