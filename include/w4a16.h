@@ -78,7 +78,8 @@ typedef enum {
 typedef enum {
     W4A16_KERNEL_AUTO = 0,    /* let the dispatch decide                                      */
     W4A16_KERNEL_GEMV = 1,    /* decode GEMV: split-K CUDA-core (plain layout, any M) or the
-                                 persistent stream-K warp-MMA kernel (tiled layout, M <= 16) */
+                                 persistent stream-K warp-MMA kernel (tiled layout, M <= 16, over
+                                 K slices when A does not fit whole) */
     W4A16_KERNEL_TC = 2       /* tcgen05 tensor-core GEMM, TMEM accumulator (tiled layout)     */
 } w4a16_kernel;
 
@@ -258,7 +259,9 @@ W4A16_API int w4a16_repack(const int32_t* codes, const void* scales, const int32
 /*
  * w4a16_workspace_bytes -- device scratch that w4a16_gemm needs for an M x N x K call, large
  * enough for any kernel the call may run: 64 KiB of per-tile counters of the stream-K decode
- * kernel, followed by split-K FP32 partial sums. Depends on the SM count of the current device.
+ * kernel, followed by FP32 partial sums (the split-K sums of the plain-layout GEMV, or the decode
+ * kernel's cut-tile sums and, when it runs over S slices of K, S x M x N FP32 slice outputs).
+ * Depends on the SM count of the current device.
  * Returns 0 only for arguments w4a16_gemm rejects.
  */
 W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
@@ -266,13 +269,16 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
 /*
  * w4a16_select_kernel -- the M-based dispatch, as a pure host function: returns the
  * w4a16_kernel that w4a16_gemm(..., W4A16_KERNEL_AUTO) runs on the tiled layout for this shape.
- * M <= 16 is bound by the weight stream and goes to the decode GEMV (W4A16_KERNEL_GEMV); larger M
+ * Small M is bound by the weight stream and goes to the decode GEMV (W4A16_KERNEL_GEMV); larger M
  * goes to the tensor-core GEMM ("INT8 vs INT4 Quantization, in depth", section "Two regimes:
  * waiting for memory, waiting for math"). The plain layout always runs the CUDA-core GEMV.
  * The environment variable W4A16_FORCE_KERNEL=gemv|tc overrides the choice.
  * On the tiled layout the decode GEMV is the persistent stream-K kernel (one CTA per SM, unit
- * records streamed by bulk copies, warp-level tensor-core MMA). When M rows of A do not fit in
- * its shared memory, W4A16_KERNEL_AUTO runs the tensor-core GEMM instead.
+ * records streamed by bulk copies, warp-level tensor-core MMA). When the M rows of A for the
+ * whole K do not fit in its shared memory it runs over S equal slices of K (one launch each,
+ * FP32 slice outputs added in order by a last kernel). AUTO takes it for M <= 8 (whole K or
+ * slices) and for 9 <= M <= 16 only when K fits whole; otherwise the tensor-core GEMM (measured:
+ * with 9-16 rows the sliced decode kernel is slower than the tensor-core GEMM).
  */
 W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
 
