@@ -236,3 +236,12 @@ def test_fp8_rejects_bad_arguments_before_any_launch(L):
     assert L.w4a16_fp8_gemm(a, b, 0, 256, c, d, 128, P(5 << 20), 0, None, None) == native.EINVAL
     assert L.w4a16_fp8_gemm(a, b, 1, 256, c, d, 128, P(5 << 20), 2, None, None) == native.EINVAL
     assert L.w4a16_fp8_gemm(a, b, 1, 256, c, P((4 << 20) + 4), 128, P(5 << 20), 0, None, None) == native.EALIGN
+
+
+def test_workspace_covers_the_k_slices_of_the_decode_kernel():
+    """16 rows of A for K = 8192 do not fit in the decode kernel's shared memory whole: the
+    workspace then also holds the FP32 outputs of its K slices (at least two of M x N x 4 B)."""
+    M, N, K = 16, 28672, 8192
+    assert native.w4a16_workspace_bytes(M, N, K, 128) >= 65536 + 2 * M * N * 4
+    # one row fits whole: counters plus the cut-tile sums only
+    assert native.w4a16_workspace_bytes(1, N, K, 128) < 65536 + M * N * 4
