@@ -102,3 +102,23 @@ def test_rank_helpers_over_two_gloo_ranks():
         assert mx == 11.5                       # the slower rank's time on every rank
     assert res[0][3] != res[1][3]               # each rank draws its own replica
     assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` times the FP64 oracle on the host cores and prints one JSON
+    line with the keys the harness reads (no GPU needed)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                         cwd=root, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
