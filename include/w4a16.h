@@ -148,7 +148,8 @@ W4A16_API size_t w4a16_gptq_workspace_bytes(int K, int N);
  *   X          device, calibration inputs [S, K] row-major, 16-bit of type x_dtype.
  *   x_dtype    W4A16_F16 or W4A16_BF16.
  *   S          calibration rows, >= 1.
- *   K, N, group, sym   as for w4a16_quantize.
+ *   K, N, group, sym   as for w4a16_quantize; K <= 29056 (the triangular inverse keeps one FP64
+ *              column of K values in shared memory), else W4A16_EUNSUPPORTED.
  *   damp       damping as a fraction of mean(diag H), added to the diagonal (0.01 is usual);
  *              >= 0 and finite.
  *   codes, scales, zeros   device out, the plain layout of w4a16_quantize (zeros NULL iff sym).

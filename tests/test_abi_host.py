@@ -197,6 +197,8 @@ def test_gptq_rejects_bad_arguments_before_any_launch(L):
     assert call(ws=None) == native.EINVAL
     assert call(wsb=need - 1) == native.EWORKSPACE
     assert call(X=P((2 << 20) + 2)) == native.EALIGN
+    big = 29056 + 128
+    assert call(K=big, wsb=L.w4a16_gptq_workspace_bytes(big, N)) == native.EUNSUPPORTED
 
 
 def test_awq_rejects_bad_arguments_before_any_launch(L):
