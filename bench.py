@@ -44,7 +44,7 @@ SYM = 0
 SWEEP_K, SWEEP_N, SWEEP_M = 8192, 28672, 256
 METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=256, as % of B200 roofline"
 # DRAM traffic (read + write) per algorithmic byte of the decode kernel, from one ncu capture of
-# the same kernel on a layer larger than L2 (profiles/gemv_stream_gate_up70b_m1.md): every unit
+# the same kernel on a layer larger than L2 (the 8192 x 57344 gate+up layer, fp16, M = 1): every unit
 # record streams once, so traffic scales with the units a launch processes.
 DECODE_TRAFFIC_RATIO = 1.017
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of gemv_stream_kernel "
