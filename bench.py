@@ -3,18 +3,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (N=1 line): the decode linears of a 32-layer Llama-3-8B-shaped model for one token,
-M = 1: per layer (K, N) = (4096, 6144) qkv, (4096, 4096) o, (4096, 28672) gate+up,
-(14336, 4096) down; g128 asymmetric INT4; fp16 activations ~ N(0, 1); weights ~ N(0, 0.02).
-Four weight matrices are drawn and quantized, and each is copied into 32 distinct device
-buffers: one step streams 3.63 GB of packed weights, so L2 (126 MB) cannot serve repeats.
-A step is the 128 GEMMs of one token, replayed from a CUDA graph.
+Workload of the headline line: the decode linears of an 80-layer Llama-3-70B-shaped model for
+one token, M = 1: per layer (K, N) = (8192, 10240) qkv, (8192, 8192) o, (8192, 57344) gate+up,
+(28672, 8192) down; g128 asymmetric INT4; bf16 activations ~ N(0, 1); weights ~ N(0, 0.02).
+Four weight matrices are drawn and quantized, and each is copied into 80 distinct device
+buffers: one step streams 35.6 GB of packed weights, so L2 (126 MB) cannot serve repeats.
+A step is the 320 GEMMs of one token, replayed from a CUDA graph.
 
 Printed (rank 0, one JSON line): value = algorithmic bytes of all ranks' steps / max-over-ranks
 device time (GB/s); e2e = the same through the Python API with the step's activations copied
-from pinned host memory and its outputs read back; roofline of the dominant kernel; the FP64
-oracle's throughput on the host cores (cpu_baseline); clocks sampled during the timed region;
-and an M = 256 measurement on the (8192, 28672) sweep layer (TFLOPS).
+from pinned host memory and its outputs read back; roofline of the dominant kernel (its in-step
+time); the FP64 oracle's throughput on the host cores (cpu_baseline); clocks sampled during the
+timed region. Extra keys: the 32-layer Llama-3-8B stack, the (8192, 28672) sweep layer at
+M = 256 (TFLOPS), the naive dequantize-then-GEMM path, the calibrated encoders, the crossover
+sweep against the W8A8 FP8 path, the format variants and the oracle on every configuration.
 
 N > 1 (torchrun): weak scaling, every rank runs its own replica of the workload; no collective
 on the data path (NCCL carries only the barrier and the max of the timings).
@@ -43,12 +45,11 @@ GROUP = 128
 SYM = 0
 SWEEP_K, SWEEP_N, SWEEP_M = 8192, 28672, 256
 METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=256, as % of B200 roofline"
-# DRAM traffic (read + write) per algorithmic byte of the decode kernel, from one ncu capture of
-# the same kernel on a layer larger than L2 (the 8192 x 57344 gate+up layer, fp16, M = 1): every unit
-# record streams once, so traffic scales with the units a launch processes.
-DECODE_TRAFFIC_RATIO = 1.017
-DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of gemv_stream_kernel "
-                         "(fp16, M=1) on the 8192x57344 layer, scaled by bytes per launch")
+SWEEP_MS = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 2048)
+# ncu DRAM traffic of the decode kernel, written by hand from a capture into this file, with the
+# hash of the kernel sources it was taken on (the bench reports it only while they match)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_stream_traffic.json")
+DECODE_SOURCES = ("gemv_stream.cu", "sm100_ptx.cuh", "tiled_layout.cuh", "common.cuh")
 
 
 # ----------------------------------------------------------------------------- work model
@@ -346,12 +347,39 @@ def time_e2e(torch, stack, steps, warmup):
     return start.elapsed_time(end) / steps
 
 
-def bench_70b(torch, native, synthetic, seed, steps, warmup, rank):
-    """GB/s of one M = 1 decode step over a Llama-3-70B-shaped linear stack: 80 layers x (qkv, o,
-    gate+up, down), g128 asymmetric INT4, bf16 activations, 35 GB of packed weights, replayed from
-    a CUDA graph; plus each shape's mean device time per launch."""
-    stack = DecodeStack(torch, native, synthetic, seed, layers=LAYERS_70B, linears=LLAMA70B_LINEARS,
-                        bf16=True)
+def decode_sources_sha():
+    """Hash of the decode kernel's sources (the files its ncu traffic capture depends on)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "weight_only_int4_07_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def decode_traffic(bytes_per_launch):
+    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu capture,
+    scaled from the captured launch to `bytes_per_launch` algorithmic bytes (the kernel streams each
+    unit record once, so its traffic grows with the units a launch processes). Returns
+    (bytes or None, provenance); None when the kernel's sources changed after the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    t = json.load(open(TRAFFIC_FILE))
+    if t.get("sources_sha") != decode_sources_sha():
+        return None, {"stale": True, "capture": t.get("capture")}
+    ratio = t["dram_bytes"] / t["algorithmic_bytes"]
+    return ratio * bytes_per_launch, {"ratio_to_algorithmic": ratio, "capture": t["capture"],
+                                      "summary": t.get("summary")}
+
+
+def time_stack(torch, native, synthetic, seed, layers, linears, bf16, steps, warmup, world, dev,
+               gpu_index, e2e=True):
+    """One decode step over a stack of linears (M = 1), replayed from a CUDA graph: device time per
+    step (max over ranks), the kernel launches in the step, each shape's isolated launch time and,
+    optionally, the end-to-end step through the Python API."""
+    stack = DecodeStack(torch, native, synthetic, seed, layers=layers, linears=linears, bf16=bf16)
+    torch.cuda.synchronize()
     for _ in range(max(warmup, 1)):
         stack.step()
     torch.cuda.synchronize()
@@ -359,17 +387,31 @@ def bench_70b(torch, native, synthetic, seed, steps, warmup, rank):
     with torch.cuda.graph(graph):
         stack.step()
     torch.cuda.synchronize()
+    kernels_per_step = count_graph_kernels(graph)
+    if hasattr(graph, "instantiate"):
+        try:
+            graph.instantiate()
+        except RuntimeError:
+            pass
     for _ in range(warmup):
         graph.replay()
-    with ClockSampler(rank) as clk:
-        ms = time_graph(torch, graph, steps, 1, None)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clk:
+        ms = time_graph(torch, graph, steps, world, dev)
+    ms_max = max_over_ranks(ms, world, dev)
     launches = time_per_launch(torch, stack, 1)
     per_shape = {name: {"K": K, "N": N, "mean_us": 1e3 * statistics.mean(v),
                         "gbs": algorithmic_bytes(1, K, N) / (statistics.mean(v) * 1e-3) / 1e9}
                  for (name, K, N), v in launches.items()}
-    out = {"ms_per_step": ms, "bytes_per_step": stack.bytes_per_step,
+    out = {"ms_per_step": ms_max, "bytes_per_step": stack.bytes_per_step,
            "weight_bytes_per_step": stack.weight_bytes, "gemms_per_step": len(stack.calls),
-           "per_shape": per_shape, "clocks": clk.summary()}
+           "kernels_per_step": kernels_per_step, "isolated_per_shape": per_shape,
+           "clocks": clk.summary(), "tiled": stack.tiled}
+    if e2e:
+        e2e_ms = max_over_ranks(time_e2e(torch, stack, steps, warmup), world, dev)
+        out["e2e"] = {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": stack.A.numel() * 2, "d2h_bytes_per_step": stack.C.numel() * 2,
+                      "ms_per_step": e2e_ms}
     del graph, stack
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -553,7 +595,7 @@ def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv",
     return out
 
 
-def bench_crossover(torch, native, synthetic, seed, Ms=(1, 4, 8, 16, 64, 128, 256, 512, 1024, 2048), reps=6):
+def bench_crossover(torch, native, synthetic, seed, Ms=SWEEP_MS, reps=6):
     """W4A16 against the W8A8 FP8 path on the (8192, 28672) sweep layer, bf16 activations, per
     batch size M: device time of one W4A16 GEMM (the library's dispatch on the tiled layout) and of
     one FP8 step (per-row activation quantization + the kind::f8f6f4 GEMM), each on two rotating
@@ -612,6 +654,78 @@ def bench_crossover(torch, native, synthetic, seed, Ms=(1, 4, 8, 16, 64, 128, 25
             "crossover_M": (min(faster) if faster else None)}
 
 
+def bench_variants(torch, native, synthetic, seed, copies=4, reps=6):
+    """The format variants: K = N = 8192, weights 0.02 * Student-t(5), symmetric and asymmetric,
+    group 32 and 128, fp16 and bf16 activations, M in {1, 16, 256}. Per variant the fused GEMM
+    (the library's dispatch on the tiled layout) and the naive path (dequantize to 16 bits, then
+    torch.matmul), mean device time over `copies` rotating weight copies (4 x 34-39 MB, more than
+    L2 holds)."""
+    dev = torch.device("cuda")
+    K = N = 8192
+    stream = torch.cuda.current_stream()
+    prev = torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction, \
+        torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = False
+    W = torch.from_numpy(synthetic.weights_student_t(K, N, seed).view(np.int16)).view(torch.float16).to(dev)
+    out = []
+    try:
+        for sym in (1, 0):
+            for group in (32, 128):
+                codes, scales, zeros = native.w4a16_quantize(W, group, sym)
+                tiled = [native.w4a16_repack(codes, scales, zeros, K, N, group, sym) for _ in range(copies)]
+                for bf16 in (False, True):
+                    tdt = torch.bfloat16 if bf16 else torch.float16
+                    Wd = torch.empty((K, N), dtype=tdt, device=dev)
+                    for M in (1, 16, 256):
+                        A = torch.from_numpy(synthetic.activations(
+                            M, K, seed + M, dtype=synthetic.BF16 if bf16 else synthetic.F16).view(np.int16)).view(
+                            tdt).to(dev)
+                        C = torch.empty((M, N), dtype=tdt, device=dev)
+                        ws = torch.zeros(max(native.w4a16_workspace_bytes(M, N, K, group), 16), dtype=torch.uint8,
+                                         device=dev)
+
+                        def fused(i):
+                            native.w4a16_gemm(A, tiled[i % copies], None, None, N, group, sym,
+                                              layout=native.LAYOUT_TILED, C=C, workspace=ws)
+
+                        def naive(i):
+                            native.w4a16_dequantize(codes, scales, zeros, K, N, group, sym, out=Wd)
+                            torch.matmul(A, Wd, out=C)
+
+                        res = {}
+                        for name, fn in (("fused", fused), ("naive", naive)):
+                            for i in range(3):
+                                fn(i)
+                            torch.cuda.synchronize()
+                            torch.cuda._sleep(int(20e6))
+                            evs = []
+                            for i in range(reps):
+                                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                                e0.record(stream)
+                                fn(i)
+                                e1.record(stream)
+                                evs.append((e0, e1))
+                            torch.cuda.synchronize()
+                            res[name] = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+                        nbytes = algorithmic_bytes(M, K, N, group=group, sym=sym)
+                        out.append({"sym": bool(sym), "group": group, "acts": "bf16" if bf16 else "fp16", "M": M,
+                                    "fused_us": res["fused"], "naive_us": res["naive"],
+                                    "fused_gbs": nbytes / (res["fused"] * 1e-6) / 1e9,
+                                    "fused_tflops": gemm_flops(M, K, N) / (res["fused"] * 1e-6) / 1e12,
+                                    "kernel": {1: "gemv", 2: "tc"}.get(native.w4a16_select_kernel(M, N, K, group))})
+                        del A, C, ws
+                    del Wd
+                del codes, scales, zeros, tiled
+                torch.cuda.empty_cache()
+    finally:
+        (torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction,
+         torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction) = prev
+    del W
+    torch.cuda.empty_cache()
+    return {"K": K, "N": N, "weights": "0.02 * Student-t(5)", "points": out}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def host_cores():
     try:
@@ -620,28 +734,34 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def oracle_prepare(synthetic, seed, threads):
-    """One Llama-3-8B-shaped layer quantized by the oracle, with one activation row per linear."""
+ORACLE_COLS = 2048   # output columns of each 70B linear in the oracle's timed sample
+
+
+def oracle_prepare(synthetic, seed, threads, linears=LLAMA70B_LINEARS, cols=ORACLE_COLS, a_dtype=1):
+    """The oracle's timed sample of the headline workload: each linear of one Llama-3-70B-shaped
+    layer restricted to its first `cols` output columns (RTN quantization is per column, so the
+    sample has the layer's per-weight work), quantized by the oracle, one bf16 activation row."""
     import oracle
 
     packed = []
-    for i, (name, K, N) in enumerate(LLAMA8B_LINEARS):
-        Wb = synthetic.weights_normal(K, N, seed + i)
+    for i, (name, K, N) in enumerate(linears):
+        n = min(N, cols)
+        Wb = synthetic.weights_normal(K, n, seed + i)
         st, c, s, z = oracle.quantize(Wb, GROUP, SYM, nthreads=threads)
-        Ab = synthetic.activations(1, K, seed + 200 + i)
-        packed.append((K, N, c, s, z, Ab))
+        Ab = synthetic.activations(1, K, seed + 200 + i, dtype=a_dtype)
+        packed.append((K, n, c, s, z, Ab, a_dtype))
     return packed
 
 
 def oracle_pass(packed, threads):
-    """One pass of the FP64 oracle over the layer's four linears (all columns, M = 1).
+    """One pass of the FP64 oracle over the sample's linears (M = 1, all sampled columns).
     Returns (algorithmic bytes, seconds)."""
     import oracle
 
     nbytes, secs = 0, 0.0
-    for (K, N, c, s, z, Ab) in packed:
+    for (K, N, c, s, z, Ab, a_dtype) in packed:
         t0 = time.perf_counter()
-        oracle.linear(Ab, 0, c, s, z, N, GROUP, SYM, nthreads=threads)
+        oracle.linear(Ab, a_dtype, c, s, z, N, GROUP, SYM, nthreads=threads)
         secs += time.perf_counter() - t0
         nbytes += algorithmic_bytes(1, K, N)
     return nbytes, secs
@@ -661,7 +781,60 @@ def oracle_sample(synthetic, seed, threads, budget_s=15.0, packed=None):
     return nbytes / total / 1e9, total, reps, packed
 
 
+ORACLE_SAMPLE = ("the four linears of one Llama-3-70B-shaped layer (8192x10240, 8192x8192, 8192x57344, "
+                 "28672x8192), first %d output columns of each, M=1, g128 asym, bf16 acts; FP64 oracle" % ORACLE_COLS)
+
+
+def oracle_configs(synthetic, threads, sub_cols=512):
+    """The FP64 oracle (quantize excluded, the layer's matmul timed) on every configuration:
+    full for the tiny layer and the Llama-3-8B linears; on the first `sub_cols` output columns of
+    each layer for the sweep, the format variants and the 70B stack, extrapolated by the column
+    count (the oracle's work is the same for every column) and labelled so."""
+    import oracle
+
+    def one(K, N, M, group, sym, a_dtype, seed, wfn=synthetic.weights_normal, cols=None):
+        n = N if cols is None else min(N, cols)
+        Wb = wfn(K, n, seed)
+        _, c, s, z = oracle.quantize(Wb, group, sym, nthreads=threads)
+        Ab = synthetic.activations(M, K, seed + 1, dtype=a_dtype)
+        t0 = time.perf_counter()
+        oracle.linear(Ab, a_dtype, c, s, z, n, group, sym, nthreads=threads)
+        return (time.perf_counter() - t0) * N / n
+
+    out = {"cores": threads, "unit": "s per GEMM"}
+    out["tiny"] = {"M": 1, "K": 512, "N": 256, "s": one(512, 256, 1, 128, 0, 0, 1)}
+    out["llama3_8b"] = {name: {"K": K, "N": N, "M": 1, "s": one(K, N, 1, GROUP, SYM, 0, 10 + i)}
+                        for i, (name, K, N) in enumerate(LLAMA8B_LINEARS)}
+    sweep = []
+    for M in SWEEP_MS:
+        t = one(SWEEP_K, SWEEP_N, M, GROUP, SYM, 1, 30, wfn=synthetic.weights_outliers, cols=sub_cols)
+        sweep.append({"M": M, "s": t, "tflops": gemm_flops(M, SWEEP_K, SWEEP_N) / t / 1e12})
+    out["sweep"] = {"K": SWEEP_K, "N": SWEEP_N, "points": sweep,
+                    "extrapolated": f"from the first {sub_cols} of {SWEEP_N} columns"}
+    var = []
+    for sym in (1, 0):
+        for group in (32, 128):
+            for a_dtype in (0, 1):
+                for M in (1, 16, 256):
+                    var.append({"sym": bool(sym), "group": group, "acts": "bf16" if a_dtype else "fp16", "M": M,
+                                "s": one(8192, 8192, M, group, sym, a_dtype, 40, wfn=synthetic.weights_student_t,
+                                         cols=sub_cols)})
+    out["variants"] = {"K": 8192, "N": 8192, "points": var,
+                       "extrapolated": f"from the first {sub_cols} of 8192 columns"}
+    stack = {}
+    for M in (1, 8, 16):
+        t = sum(one(K, N, M, GROUP, SYM, 1, 50 + i, cols=sub_cols) for i, (_, K, N) in enumerate(LLAMA70B_LINEARS))
+        stack[str(M)] = {"s_per_step": t * LAYERS_70B}
+    out["llama3_70b_stack"] = {"layers": LAYERS_70B, "per_M": stack,
+                               "extrapolated": f"one layer, first {sub_cols} columns of each linear, x{LAYERS_70B} layers"}
+    return out
+
+
 # ----------------------------------------------------------------------------- arms
+HEADLINE_WORKLOAD = ("llama3-70b decode linears (qkv 8192x10240, o 8192x8192, gate+up 8192x57344, "
+                     "down 28672x8192), M=1, g128 asym INT4, bf16 acts, 80 layers per step")
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -679,15 +852,12 @@ def run_reference(args):
         tot_s += t
     value = tot_b / tot_s / 1e9
     ms = 1e3 * tot_s / args.steps
-    sample = ("one Llama-3-8B-shaped layer per step: the four decode linears (4096x6144, 4096x4096, "
-              "4096x28672, 14336x4096), all columns, M=1, g128 asym, fp16; FP64 oracle")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama3-8b decode linears, M=1, g128 asym INT4, fp16 acts",
-                       "layers_per_step": 1},
+            "config": {"workload": HEADLINE_WORKLOAD, "sample_per_step": ORACLE_SAMPLE},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": ORACLE_SAMPLE + ", one pass per step"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -717,156 +887,109 @@ def run_ours(args):
     native.lib()
     peaks = load_peaks()
 
-    seed = replica_seed(1000, rank)
-    stack = DecodeStack(torch, native, synthetic, seed)
-    torch.cuda.synchronize()
-
-    # warm-up, then capture one step in a CUDA graph
-    for _ in range(max(args.warmup, 1)):
-        stack.step()
-    torch.cuda.synchronize()
-    graph = new_graph(torch)
-    with torch.cuda.graph(graph):
-        stack.step()
-    torch.cuda.synchronize()
-    kernels_per_step = count_graph_kernels(graph)
-    if hasattr(graph, "instantiate"):
-        try:
-            graph.instantiate()
-        except RuntimeError:
-            pass
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-
-    with ClockSampler(local_rank) as clk:
-        ms = time_graph(torch, graph, args.steps, world, dev)
-    ms_max = max_over_ranks(ms, world, dev)
-    value = world * stack.bytes_per_step / (ms_max * 1e-3) / 1e9
-
-    # per-launch device durations (roofline of the dominant kernel)
-    launches = time_per_launch(torch, stack, max(1, min(args.steps, 5)))
-    tot_bytes = sum(algorithmic_bytes(1, K, N) * len(v) for (name, K, N), v in launches.items())
-    tot_ms = sum(sum(v) for v in launches.values())
-    n_launch = sum(len(v) for v in launches.values())
-    per_shape = {name: {"K": K, "N": N, "mean_us": 1e3 * statistics.mean(v),
-                        "gbs": algorithmic_bytes(1, K, N) / (statistics.mean(v) * 1e-3) / 1e9}
-                 for (name, K, N), v in launches.items()}
-    achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
-    kernel = native.w4a16_select_kernel(1, 4096, 4096, GROUP)
-    # the decode kernel's code changed after its last ncu capture (K-slice addressing, unused at
-    # this workload's shapes), so the measured traffic is reported as a note, not as `traffic`
-    traffic = None
+    # the headline: one decode step over the 70B-shaped stack
+    r = time_stack(torch, native, synthetic, replica_seed(7000, rank), LAYERS_70B, LLAMA70B_LINEARS, True,
+                   args.steps, args.warmup, world, dev, local_rank)
+    ms_max = r["ms_per_step"]
+    value = world * r["bytes_per_step"] / (ms_max * 1e-3) / 1e9
+    # every launch of the step is the decode kernel (M = 1 on the tiled layout), so its mean
+    # in-step duration is the step's device time over its launches
+    n_launch = r["gemms_per_step"]
+    kernel = native.w4a16_select_kernel(1, 8192, 8192, GROUP) if r["tiled"] else native.KERNEL_GEMV
+    bytes_per_launch = r["bytes_per_step"] / n_launch
+    launch_us = 1e3 * ms_max / n_launch
+    achieved = bytes_per_launch / (launch_us * 1e-6) / 1e9
+    traffic, traffic_src = decode_traffic(bytes_per_launch) if r["tiled"] else (None, None)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "traffic_source": None,
-                "traffic_last_capture": {"bytes_per_launch": DECODE_TRAFFIC_RATIO * tot_bytes / n_launch,
-                                         "ratio_to_algorithmic": DECODE_TRAFFIC_RATIO,
-                                         "source": DECODE_TRAFFIC_SOURCE} if stack.tiled else None,
-                "kernel": {1: "gemv", 2: "tc"}.get(kernel, str(kernel)),
-                "bytes_per_launch": tot_bytes / n_launch, "launch_us": 1e3 * tot_ms / n_launch,
-                "peak_source": peaks["source"], "per_shape": per_shape}
+                "kernel": "gemv_stream_kernel" if kernel == native.KERNEL_GEMV and r["tiled"] else
+                {1: "gemv", 2: "tc"}.get(kernel, str(kernel)),
+                "bytes_per_launch": bytes_per_launch, "launch_us_in_step": launch_us,
+                "launches_per_step": n_launch, "peak_source": peaks["source"] + " (copy)",
+                "traffic_source": traffic_src, "isolated_per_shape": r["isolated_per_shape"]}
 
-    # end to end through the Python API, pinned host <-> device copies inside the timed region
-    e2e_ms = time_e2e(torch, stack, args.steps, args.warmup)
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
-    e2e = {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-           "h2d_bytes_per_step": stack.A.numel() * 2, "d2h_bytes_per_step": stack.C.numel() * 2,
-           "ms_per_step": e2e_ms}
-
-    del graph
-    torch.cuda.synchronize()
-    gemms_per_step = len(stack.calls)
-    layout = "tiled" if stack.tiled else "plain"
-    weight_bytes = stack.weight_bytes
-    bytes_per_step = stack.bytes_per_step
-
-    del stack
-    torch.cuda.empty_cache()
-
-    # the same metric over the 70B-shaped stack (the layers the ">= 75% of HBM" target names)
-    m1_70b = None
-    if not args.skip_70b:
-        r70 = bench_70b(torch, native, synthetic, replica_seed(7000, rank), max(2, min(args.steps, 10)),
-                        args.warmup, local_rank)
-        ms70 = max_over_ranks(r70["ms_per_step"], world, dev)
-        gbs70 = world * r70["bytes_per_step"] / (ms70 * 1e-3) / 1e9
-        m1_70b = {"value": gbs70, "unit": "GB/s", "ms_per_step": ms70,
-                  "frac": gbs70 / world / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
-                  "peak_source": peaks["source"], "per_shape": r70["per_shape"], "clocks": r70["clocks"],
-                  "config": {"workload": "llama3-70b decode linears (qkv 8192x10240, o 8192x8192, "
-                                         "gate+up 8192x57344, down 28672x8192), M=1, g128 asym INT4, "
-                                         "bf16 acts, 80 layers per step",
-                             "gemms_per_step": r70["gemms_per_step"],
-                             "weight_bytes_per_step": r70["weight_bytes_per_step"],
-                             "algorithmic_bytes_per_step": r70["bytes_per_step"]}}
+    # the 32-layer Llama-3-8B stack (the smaller decode configuration)
+    m1_8b = None
+    if not args.skip_8b:
+        r8 = time_stack(torch, native, synthetic, replica_seed(1000, rank), LAYERS, LLAMA8B_LINEARS, False,
+                        args.steps, args.warmup, world, dev, local_rank, e2e=False)
+        gbs8 = world * r8["bytes_per_step"] / (r8["ms_per_step"] * 1e-3) / 1e9
+        m1_8b = {"value": gbs8, "unit": "GB/s", "ms_per_step": r8["ms_per_step"],
+                 "frac": gbs8 / world / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                 "isolated_per_shape": r8["isolated_per_shape"], "clocks": r8["clocks"],
+                 "config": {"workload": "llama3-8b decode linears (qkv 4096x6144, o 4096x4096, gate+up "
+                                        "4096x28672, down 14336x4096), M=1, g128 asym INT4, fp16 acts, "
+                                        "32 layers per step",
+                            "gemms_per_step": r8["gemms_per_step"],
+                            "algorithmic_bytes_per_step": r8["bytes_per_step"]}}
 
     # M = 256 on the sweep layer (TFLOPS)
     m256 = None
     if not args.skip_m256:
-        r = bench_m256(torch, native, synthetic, replica_seed(5000, rank), max(2, min(args.steps, 10)),
-                       args.warmup)
-        ms256 = max_over_ranks(r["ms"], world, dev)
-        tf = gemm_flops(r["M"], r["K"], r["N"]) / (ms256 * 1e-3) / 1e12
+        rm = bench_m256(torch, native, synthetic, replica_seed(5000, rank), max(2, min(args.steps, 10)),
+                        args.warmup)
+        ms256 = max_over_ranks(rm["ms"], world, dev)
+        tf = gemm_flops(rm["M"], rm["K"], rm["N"]) / (ms256 * 1e-3) / 1e12
         peak_tf = peaks["bf16_tflops"]
-        m256 = {"value": world * tf, "unit": "TFLOP/s", "ms": ms256, "kernel": r["kernel"],
+        m256 = {"value": world * tf, "unit": "TFLOP/s", "ms": ms256, "kernel": rm["kernel"],
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
-                             "frac": tf / peak_tf, "traffic": None, "peak_source": peaks["source"] +
-                             " burst"},
-                "config": {"M": r["M"], "K": r["K"], "N": r["N"], "group": GROUP, "sym": False,
+                             "frac": tf / peak_tf, "traffic": None,
+                             "peak_source": peaks["source"] + " burst"},
+                "config": {"M": rm["M"], "K": rm["K"], "N": rm["N"], "group": GROUP, "sym": False,
                            "acts": "bf16", "weights": "N(0,0.02) with 0.1% outliers x20",
                            "l2": "4 rotating weight copies of 122 MB"}}
 
-    # the naive path (dequantize to 16 bits, then the library GEMM) on the same shapes
     naive = None
     if not args.skip_naive:
         naive = bench_naive(torch, native, synthetic, replica_seed(9000, rank), max(2, min(args.steps, 10)),
                             args.warmup)
-        for name, r in naive.items():
-            fused_us = (roofline["per_shape"][name]["mean_us"] if name in roofline["per_shape"]
-                        else (1e3 * m256["ms"] if (name == "sweep_m256" and m256) else None))
-            r["fused_us"] = fused_us
-            r["fused_speedup"] = None if fused_us is None else r["total_us"] / fused_us
+        fused = dict(m1_8b["isolated_per_shape"]) if m1_8b else {}
+        for name, rr in naive.items():
+            us = (fused[name]["mean_us"] if name in fused
+                  else (1e3 * m256["ms"] if (name == "sweep_m256" and m256) else None))
+            rr["fused_us"] = us
+            rr["fused_speedup"] = None if us is None else rr["total_us"] / us
 
-    # the calibrated encoders (offline), per 8B layer shape
     encoders = None
     if not args.skip_encoders:
         encoders = bench_encoders(torch, native, synthetic, replica_seed(9500, rank))
 
-    # W4A16 against the W8A8 FP8 path across batch sizes (the crossover)
     crossover = None
     if not args.skip_crossover:
         crossover = bench_crossover(torch, native, synthetic, replica_seed(9700, rank))
 
+    variants = None
+    if not args.skip_variants:
+        variants = bench_variants(torch, native, synthetic, replica_seed(9800, rank))
+
     cpu = None
+    oracle_all = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         threads = host_cores()
         gbs, secs, reps, packed = oracle_sample(synthetic, 11, threads, budget_s=args.cpu_budget)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"{reps} pass(es) over one Llama-3-8B-shaped layer (4 decode linears, all "
-                         f"columns, M=1, g128 asym, fp16), FP64 oracle, {secs:.1f} s"}
-        # the same oracle on one host thread (one pass)
+               "sample": f"{reps} pass(es) over " + ORACLE_SAMPLE + f", {secs:.1f} s"}
         gbs1, secs1, _, _ = oracle_sample(synthetic, 11, 1, budget_s=0.0, packed=packed)
         cpu["single_thread"] = {"value": gbs1, "unit": "GB/s", "cores": 1, "seconds": secs1}
+        if not args.skip_oracle_configs:
+            oracle_all = oracle_configs(synthetic, threads)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-                "data": "synthetic (seeded; weights N(0,0.02) fp16, activations N(0,1) fp16)",
-                "config": {"workload": "llama3-8b decode linears (qkv 4096x6144, o 4096x4096, "
-                                       "gate+up 4096x28672, down 14336x4096), M=1, g128 asym INT4, "
-                                       "fp16 acts, 32 layers per step",
-                           "layers": LAYERS, "gemms_per_step": gemms_per_step,
-                           "weight_bytes_per_step": weight_bytes,
-                           "algorithmic_bytes_per_step": bytes_per_step,
-                           "parallelism": f"replica x{world}", "layout": layout,
-                           "l2": "inputs larger than L2: 3.63 GB of packed weights per step",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded; weights N(0,0.02) fp16, activations N(0,1) bf16)",
+                "config": {"workload": HEADLINE_WORKLOAD, "layers": LAYERS_70B,
+                           "gemms_per_step": r["gemms_per_step"],
+                           "weight_bytes_per_step": r["weight_bytes_per_step"],
+                           "algorithmic_bytes_per_step": r["bytes_per_step"],
+                           "parallelism": f"replica x{world}", "layout": "tiled" if r["tiled"] else "plain",
+                           "l2": "inputs larger than L2: 35.6 GB of packed weights per step",
                            "timing": "CUDA graph replay of one step, CUDA events"},
-                "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk.summary(),
-                "gpu_launches": (None if kernels_per_step is None else kernels_per_step * args.steps),
-                "m1_70b": m1_70b, "m256": m256, "naive": naive, "encoders": encoders,
-                "crossover": crossover}
+                "e2e": r["e2e"], "roofline": roofline, "cpu_baseline": cpu, "clocks": r["clocks"],
+                "gpu_launches": (None if r["kernels_per_step"] is None else r["kernels_per_step"] * args.steps),
+                "m1_8b": m1_8b, "m256": m256, "naive": naive, "encoders": encoders,
+                "crossover": crossover, "variants": variants, "oracle_configs": oracle_all}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -911,7 +1034,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--skip-m256", action="store_true")
-    ap.add_argument("--skip-70b", action="store_true")
+    ap.add_argument("--skip-8b", action="store_true")
+    ap.add_argument("--skip-variants", action="store_true")
+    ap.add_argument("--skip-oracle-configs", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-naive", action="store_true")
     ap.add_argument("--skip-encoders", action="store_true")

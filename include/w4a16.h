@@ -334,9 +334,9 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
  *   - Every call on a device uses the same array, which keeps the last call's contents (nothing
  *     in it needs to start at zero). Calls that can overlap on the GPU -- on different streams,
  *     or from different host threads -- race on it: order them on one stream.
- *   - The first call on each device looks up the array's device address with
- *     cudaGetSymbolAddress (with that device current); make that first call before any stream
- *     capture begins.
+ *   - Every call looks up the array's device address with cudaGetSymbolAddress (with the
+ *     caller's device current); the first call on a device also loads the library's device code
+ *     there, so make that first call before any stream capture begins.
  * Arguments as w4a16_gemm with layout W4A16_LAYOUT_PLAIN (codes [K/8, N], scales [K/g, N],
  * zeros [K/g, N/8] or NULL when sym), without workspace, kernel choice or dev_status.
  * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
@@ -345,6 +345,19 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
 W4A16_API int w4a16_gemm_noalloc(const void* A, int a_dtype, int M, int K, const int32_t* codes,
                                  const void* scales, const int32_t* zeros, int N, int group, int sym,
                                  void* C, void* stream);
+
+/*
+ * w4a16_set_wait_limit_ns -- the time limit of every bounded wait inside the library's kernels
+ *   (a pipeline barrier, or a counter another CTA of the same launch sets), in nanoseconds, for
+ *   launches made after the call; 0 restores the default of 2 s. Returns the previous limit.
+ *   A wait that runs out makes the kernel record W4A16_ETIMEOUT in dev_status, stop issuing work,
+ *   let its copies and MMAs in flight complete, free its tensor memory and return, so the device
+ *   stays usable; its outputs are then unspecified and its workspace must be zeroed again. A very
+ *   short limit (say 1 ns) makes the waits run out on purpose, which is how the timeout path is
+ *   tested. Not on the pages: a property of this library. Process-wide; safe to call from any
+ *   thread (each launch reads the value once).
+ */
+W4A16_API uint64_t w4a16_set_wait_limit_ns(uint64_t ns);
 
 /* w4a16_status_str -- a static, human-readable name for a status code. */
 W4A16_API const char* w4a16_status_str(int status);

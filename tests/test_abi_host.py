@@ -247,3 +247,43 @@ def test_workspace_covers_the_k_slices_of_the_decode_kernel():
     assert native.w4a16_workspace_bytes(M, N, K, 128) >= 65536 + 2 * M * N * 4
     # one row fits whole: counters plus the cut-tile sums only
     assert native.w4a16_workspace_bytes(1, N, K, 128) < 65536 + M * N * 4
+
+
+def test_wait_limit_setter_is_host_only(L):
+    """w4a16_set_wait_limit_ns returns the previous limit; 0 restores the 2 s default."""
+    prev = native.w4a16_set_wait_limit_ns(12345)
+    assert native.w4a16_set_wait_limit_ns(0) == 12345
+    assert native.w4a16_set_wait_limit_ns(prev) == 2_000_000_000
+
+
+def _in_child(env, code):
+    import subprocess
+    import sys
+
+    e = dict(os.environ)
+    e.update(env)
+    return subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=e, capture_output=True, text=True,
+                          timeout=300)
+
+
+def test_force_kernel_environment_overrides_the_dispatch(L):
+    """W4A16_FORCE_KERNEL=gemv|tc (read once per process) replaces the M-based choice."""
+    code = ("from weight_only_int4_07_b200 import native; "
+            "print(native.w4a16_select_kernel(1, 4096, 4096, 128), native.w4a16_select_kernel(512, 4096, 4096, 128))")
+    for value, expect in (("tc", "2 2"), ("gemv", "1 1"), ("", "1 2")):
+        r = _in_child({"W4A16_FORCE_KERNEL": value}, code)
+        assert r.returncode == 0, r.stderr
+        assert r.stdout.split() == expect.split(), value
+
+
+def test_log_environment_prints_the_dispatch(L):
+    """W4A16_LOG=1 prints one line per w4a16_gemm call with the shape and the kernel chosen,
+    before any launch (here the call then fails on the host without a device: no compute)."""
+    code = ("import ctypes; from weight_only_int4_07_b200 import native; L = native.lib(); "
+            "p = ctypes.c_void_p(1 << 20); "
+            "L.w4a16_gemm(p, 0, 1, 256, p, 1, None, None, 256, 128, 0, p, p, 1 << 30, 0, None, None)")
+    r = _in_child({"W4A16_LOG": "1", "CUDA_VISIBLE_DEVICES": ""}, code)
+    assert r.returncode == 0, r.stderr
+    assert "[w4a16] gemm M=1 N=256 K=256 g=128 sym=0 layout=1 -> gemv" in r.stderr
+    r = _in_child({"W4A16_LOG": "0", "CUDA_VISIBLE_DEVICES": ""}, code)
+    assert "[w4a16]" not in r.stderr

@@ -323,16 +323,71 @@ def test_gemm_tc_unit_rows_return_dequantized_rows(a_dtype, sym):
     assert np.array_equal(got, expect)
 
 
-@pytest.mark.parametrize("M", [32, 64, 256, 512])
-def test_gemm_tc_sweep_shape_sampled(M):
-    """The (8192, 28672) sweep layer in the launch configuration the benchmark times."""
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 64, 128, 256])
+def test_gemm_sweep_shape_all_columns(M):
+    """The (8192, 28672) sweep layer in the launch configuration the benchmark times (tiled
+    layout, AUTO dispatch, one workspace reused as the benchmark does): every output element
+    against the oracle."""
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 6000 + M, a_dtype)
-    cols = synthetic.column_sample(N, 96, seed=M + 1)
+    ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED, workspace=ws,
+                          dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+    assert torch.count_nonzero(ws[:65536]).item() == 0
+
+
+@pytest.mark.parametrize("M", [512, 2048])
+def test_gemm_tc_sweep_shape_sampled(M):
+    """The sweep layer at the large-M points: 2 and 8 row blocks of 256 per channel tile; a
+    sample of columns (the FP64 oracle of all 28672 would take minutes), always including the
+    first and last channel tile."""
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
+    Ab, A = _acts(M, K, 6000 + M, a_dtype)
+    cols = np.unique(np.concatenate([synthetic.column_sample(N, 96, seed=M + 1), np.arange(128),
+                                     np.arange(N - 128, N)]))
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+
+
+TC_STREAM = [
+    # M, K, N, group, sym, a_dtype     (units = N/128 * ceil(M/BN) * K/128 against one CTA per SM)
+    (17, 8192, 256, 128, 0, 1),        # 2 tiles x 64 units < 148: one unit per CTA, tiles cut 64 ways
+    (32, 4096, 1280, 64, 1, 0),        # 320 units: tiles cut in two or three
+    (64, 2048, 9600, 128, 0, 1),       # 1200 units, about 8 per CTA
+    (100, 1024, 2048, 32, 0, 0),
+    (128, 3072, 640, 128, 1, 1),       # 5 tiles x 24 units: every tile cut among about 30 CTAs
+    (256, 2048, 1024, 64, 0, 1),
+    (600, 1024, 512, 128, 0, 1),       # three row blocks of 256 (the last ragged) per channel tile
+    (9, 8192, 1024, 128, 0, 0),        # 9 rows forced onto the tensor cores
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", TC_STREAM)
+def test_gemm_tc_stream_full_output(M, K, N, group, sym, a_dtype):
+    """The stream-K tensor-core kernel: full output within the bound, counters left at zero, and
+    a second call on the same workspace bit-identical (the cut tiles are summed in CTA order)."""
+    kind = "student_t" if sym else "outliers"
+    Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 130 + K + N)
+    Ab, A = _acts(M, K, 1600 + M, a_dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                          kernel=native.KERNEL_TC, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
+    assert torch.count_nonzero(ws[:65536]).item() == 0
+    C2 = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
+                           kernel=native.KERNEL_TC, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(C.view(torch.int16), C2.view(torch.int16))
 
 
 @pytest.mark.parametrize("sym,group,a_dtype", [(s, g, d) for s in (0, 1) for g in (32, 128) for d in (0, 1)])
@@ -364,16 +419,15 @@ DECODE_GEMM = [
 
 
 @pytest.mark.parametrize("K,N", LLAMA8B)
-def test_gemm_llama8b_decode_tiled_sampled(K, N):
+def test_gemm_llama8b_decode_tiled_all_columns(K, N):
     """The four Llama-3-8B decode layers at M = 1 in the launch configuration of the benchmark
-    (tiled layout, AUTO dispatch)."""
+    (tiled layout, AUTO dispatch): every output column."""
     group, sym, a_dtype = 128, 0, 0
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 1000 + N)
     Ab, A = _acts(1, K, 2000 + K, a_dtype)
-    cols = synthetic.column_sample(N, 512, seed=K + N + 1)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
 @pytest.mark.parametrize("M,K,N,group,sym,a_dtype", DECODE_GEMM)
@@ -388,16 +442,15 @@ def test_gemm_gemv_mma_full_output(M, K, N, group, sym, a_dtype):
     _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
-@pytest.mark.parametrize("M", [1, 2, 4])
-def test_gemm_gemv_mma_sweep_shape_sampled(M):
+@pytest.mark.parametrize("M", [2, 4])
+def test_gemm_gemv_mma_sweep_shape_all_columns(M):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9700 + M, a_dtype)
-    cols = synthetic.column_sample(N, 96, seed=M + 4)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED,
                           kernel=native.KERNEL_GEMV)
     torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
 # ----------------------------------------------------------------------------- stream-K decode GEMV
@@ -506,30 +559,30 @@ def test_gemm_stream_bf16_rows_outside_fp16_range(sym):
         _check_gemm(C, Ab, 1, oc, os_, oz, N, group, sym, out_rel=2.0 ** -8)
 
 
+@pytest.mark.parametrize("M", [1, 8, 16])
 @pytest.mark.parametrize("K,N", [(8192, 10240), (8192, 8192), (8192, 57344), (28672, 8192)])
-def test_gemm_stream_llama70b_decode_sampled(K, N):
-    """The Llama-3-70B-shaped layers at M = 1 (bf16), sampled columns."""
+def test_gemm_llama70b_decode_all_columns(K, N, M):
+    """The Llama-3-70B-shaped layers (bf16) at the stack's batch sizes, in the launch
+    configuration of the benchmark (tiled layout, AUTO dispatch): every output element."""
     group, sym, a_dtype = 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 3000 + N)
-    Ab, A = _acts(1, K, 4000 + K, a_dtype)
-    cols = synthetic.column_sample(N, 256, seed=K + N + 7)
+    Ab, A = _acts(M, K, 4000 + K + M, a_dtype)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
-@pytest.mark.parametrize("M", [6, 8, 9, 16])
-def test_gemm_auto_sweep_shape_sampled_skinny(M):
+@pytest.mark.parametrize("M", [6, 9])
+def test_gemm_auto_sweep_shape_skinny_all_columns(M):
     """M rows of A too long to sit in the decode kernel's shared memory whole: the AUTO dispatch
-    runs the decode kernel over K slices (one launch each, FP32 outputs added in slice order),
-    still within the bound."""
+    runs the decode kernel over K slices (one launch each, FP32 outputs added in slice order) or
+    the tensor-core kernel, every output within the bound."""
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
     Ab, A = _acts(M, K, 9900 + M, a_dtype)
-    cols = synthetic.column_sample(N, 96, seed=M + 5)
     C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED)
     torch.cuda.synchronize()
-    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    _check_gemm(C, Ab, a_dtype, oc, os_, oz, N, group, sym)
 
 
 @pytest.mark.parametrize("M,K,N,group,sym,a_dtype", [

@@ -1,0 +1,75 @@
+"""The bounded device waits run out on purpose, and the device stays usable.
+
+Every wait inside the kernels (a pipeline barrier, or a tile counter that another CTA of the
+same launch sets) gives up after a time limit. w4a16_set_wait_limit_ns(1) shortens that limit to
+1 ns, so the first wait that is not already satisfied gives up: the kernel records W4A16_ETIMEOUT
+in dev_status, stops issuing, lets its copies and MMAs in flight complete, frees its tensor memory
+and returns. Nothing here faults, traps or spins without a limit. The test then restores the
+default limit, zeroes the workspace again (the header asks for that after a timeout) and checks
+that the next call on the same device is exact against the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_int4_07_b200 import native, synthetic
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from weight_only_int4_07_b200 import build
+
+    build.build()
+    native.lib()
+    torch.cuda.set_device(0)
+    yield
+    native.w4a16_set_wait_limit_ns(0)
+
+
+def _layer(K, N, group, sym, seed):
+    Wb = synthetic.weights_normal(K, N, seed)
+    st, oc, os_, oz = oracle.quantize(Wb, group, sym)
+    W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
+    gc, gs, gz = native.w4a16_quantize(W, group, sym)
+    return (oc, os_, oz), native.w4a16_repack(gc, gs, gz, K, N, group, sym)
+
+
+@pytest.mark.parametrize("M,kernel", [(1, native.KERNEL_GEMV), (8, native.KERNEL_GEMV),
+                                      (64, native.KERNEL_TC), (256, native.KERNEL_TC)])
+def test_waits_run_out_then_the_device_recovers(M, kernel):
+    K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
+    (oc, os_, oz), tiled = _layer(K, N, group, sym, 21)
+    Ab = synthetic.activations(M, K, 22 + M, dtype=a_dtype)
+    A = torch.from_numpy(Ab.view(np.int16)).view(torch.bfloat16).cuda()
+    ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    prev = native.w4a16_set_wait_limit_ns(1)
+    try:
+        native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED, kernel=kernel,
+                          workspace=ws, dev_status=status)
+        torch.cuda.synchronize()            # the launch returned: no wait was left without a limit
+    finally:
+        native.w4a16_set_wait_limit_ns(prev)
+    assert int(status.item()) == native.ETIMEOUT
+    # the device still works: the same call with the default limit, on a zeroed workspace
+    ws.zero_()
+    status.zero_()
+    C = native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED, kernel=kernel,
+                          workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    cols = synthetic.column_sample(N, 256, seed=M)
+    Y, Yabs = oracle.linear(Ab, a_dtype, oc, os_, oz, N, group, sym, cols=cols)
+    y = oracle.decode16(C.view(torch.int16).cpu().numpy().view(np.uint16), a_dtype)[:, cols]
+    assert np.all(np.abs(y - Y) <= REL * Yabs + ABS)
+    assert torch.count_nonzero(ws[:65536]).item() == 0
+
+

@@ -5,9 +5,11 @@ application that owns every device allocation, or a latency-critical loop that m
 cudaMalloc because it can block and synchronise the device. For them the library keeps the
 split-K partial sums in one static device array. This test calls that entry point through the
 C ABI twice in a row -- the second call finds the first call's partial sums still in the shared
-array -- and checks both outputs against w4a16_gemm's, within the bound the parity tests use.
-It also checks that a call needing more than the static array holds is refused. It lives in a
-file of its own, collected last, and passes alone in a fresh process as well.
+array -- and checks both outputs against the FP64 oracle's layer output within the acceptance
+bound, and against w4a16_gemm's output within the same bound. One case has more than 16 rows,
+so the entry point runs its 16-row chunks one after another on the shared array. It also checks
+that a call needing more than the static array holds is refused. It lives in a file of its own,
+collected last, and passes alone in a fresh process as well.
 """
 import ctypes
 
@@ -38,7 +40,8 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", [(1, 4096, 6144, 128, 0, 0), (5, 2048, 1032, 32, 1, 1)])
+@pytest.mark.parametrize("M,K,N,group,sym,a_dtype", [(1, 4096, 6144, 128, 0, 0), (5, 2048, 1032, 32, 1, 1),
+                                                     (20, 2048, 1032, 128, 0, 1)])
 def test_noalloc_matches_gemm_on_two_calls(M, K, N, group, sym, a_dtype):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
@@ -48,6 +51,7 @@ def test_noalloc_matches_gemm_on_two_calls(M, K, N, group, sym, a_dtype):
     W = torch.from_numpy(Wb.view(np.int16)).view(torch.float16).cuda()
     codes, scales, zeros = native.w4a16_quantize(W, group, sym)
     st, oc, os_, oz = oracle.quantize(Wb, group, sym)
+    assert np.array_equal(codes.cpu().numpy(), oc)   # the oracle's output below is for these weights
     tdt = torch.float16 if a_dtype == 0 else torch.bfloat16
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
@@ -59,10 +63,11 @@ def test_noalloc_matches_gemm_on_two_calls(M, K, N, group, sym, a_dtype):
                                   sym, _p(C), stream)
         assert rc == native.OK, native.status_str(rc)
         torch.cuda.synchronize()
-        _, Yabs = oracle.linear(Ab, a_dtype, oc, os_, oz, N, group, sym)
+        Y, Yabs = oracle.linear(Ab, a_dtype, oc, os_, oz, N, group, sym)
         y = C.double().cpu().numpy()
         y_ref = ref.double().cpu().numpy()
-        assert np.all(np.abs(y - y_ref) <= REL * Yabs + ABS), f"call {call}"
+        assert np.all(np.abs(y - Y) <= REL * Yabs + ABS), f"call {call}: outside the bound of the oracle"
+        assert np.all(np.abs(y - y_ref) <= REL * Yabs + ABS), f"call {call}: differs from w4a16_gemm"
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch():

@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -35,6 +36,15 @@ int forced_kernel() {
     });
     return forced;
 }
+
+}  // namespace
+
+// The limit of every bounded device wait, read by each launch (w4a16_set_wait_limit_ns).
+static std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+uint64_t w4a16::wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
+namespace {
 
 bool log_enabled() {
     static bool on = false;
@@ -73,7 +83,12 @@ int dispatch(int M, int N, int K, int group) {
 
 extern "C" {
 
-W4A16_API int w4a16_version(void) { return 100; }
+W4A16_API int w4a16_version(void) { return 200; }
+
+W4A16_API uint64_t w4a16_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns == 0 ? 2000000000ull : ns;
+    return g_wait_limit_ns.exchange(v, std::memory_order_relaxed);
+}
 
 W4A16_API const char* w4a16_status_str(int status) {
     switch (status) {
@@ -226,7 +241,9 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group) {
     int n_sm = gemv_stream_sm_count();
     if (n_sm <= 0) n_sm = 148;
     const GemvStreamPlan q = plan_gemv_stream(M, N, K, group, 0, n_sm);   // asymmetric: the larger plan
-    const size_t rest = q.ok && q.partial_bytes > p.ws_bytes ? q.partial_bytes : p.ws_bytes;
+    size_t rest = q.ok && q.partial_bytes > p.ws_bytes ? q.partial_bytes : p.ws_bytes;
+    const TcPlan t = plan_gemm_tc(M, N, K, group, 0, n_sm);
+    if (t.ok && t.partial_bytes > rest) rest = t.partial_bytes;
     return kGemvStreamCounterBytes + rest;
 }
 
@@ -281,11 +298,11 @@ W4A16_API int w4a16_gemm(const void* A, int a_dtype, int M, int K, const void* w
         st = launch_gemv_stream(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
         // M > 16, or M rows of A too long for shared memory: the tensor-core kernel
         if (st == W4A16_EUNSUPPORTED && kernel == W4A16_KERNEL_AUTO)
-            return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
+            return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
         return st;
     }
     if (chosen == W4A16_KERNEL_TC && layout == W4A16_LAYOUT_TILED) {
-        return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, dev_status, s);
+        return launch_gemm_tc(A, a_dtype, M, K, wq, N, group, sym, C, workspace, dev_status, s);
     }
     return W4A16_EUNSUPPORTED;
 }

@@ -79,8 +79,6 @@ int launch_gemv_plain(const void* A, int a_dtype, int M, int K, const int32_t* c
                       const void* scales, const int32_t* zeros, int N, int group, int sym, void* C,
                       void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
-int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
-                   void* C, int* dev_status, cudaStream_t stream);
 
 // Persistent stream-K decode kernel. Its workspace starts with one int counter per 128-channel
 // tile (kGemvStreamCounterBytes, zero between calls; each call leaves them zero), followed by
@@ -99,5 +97,25 @@ GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_s
 int gemv_stream_sm_count();
 int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
                        void* C, void* workspace, int* dev_status, cudaStream_t stream);
+
+// Persistent stream-K tensor-core GEMM. Its workspace is the same tile counters (one int per tile
+// of 128 channels x BN rows), followed by the FP32 sums of tiles cut between CTAs ([P][BN][128]).
+struct TcPlan {
+    bool ok;
+    int bn;               // rows of A per tile (the MMA's N)
+    int mblocks;          // tiles of BN rows
+    int ctas;             // persistent CTAs (one per SM)
+    int nr, na, nd;       // ring depths: record slots, activation tiles, weight tiles
+    uint32_t slot_w, off_a, off_w, off_bar;
+    size_t smem;
+    size_t partial_bytes; // workspace after the counters
+};
+TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm);
+int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
+                   void* C, void* workspace, int* dev_status, cudaStream_t stream);
+
+// Limit of every bounded wait on the device, in nanoseconds (2 s unless w4a16_set_wait_limit_ns
+// changed it); each launch reads it once.
+uint64_t wait_limit_ns();
 
 }  // namespace w4a16

@@ -9,10 +9,8 @@
 // CUDA driver reserves on every GPU that loads the library and keeps until the process exits.
 //
 // Nothing here calls cudaMalloc, cudaFree or any allocating routine. The array's name is only a
-// host-side stand-in in host code; its device address is looked up once per device, with that
-// device current, by cudaGetSymbolAddress, and passed to the kernels.
-#include <mutex>
-
+// host-side stand-in in host code; its device address is looked up by cudaGetSymbolAddress, with
+// the caller's device current, on every call, and passed to the kernels.
 #include "common.cuh"
 
 namespace w4a16 {
@@ -24,22 +22,14 @@ constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (looked up on first use).
+// Device address of g_noalloc_scratch on the current device. Looked up on every call (a cheap
+// runtime query): a cached address would go stale if the device's primary context were
+// destroyed and created again (cudaDeviceReset), since the module, and the array with it, is
+// then loaded anew and may land elsewhere.
 int scratch_on_current_device(void** addr) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ECUDA;
-    if (dev < 0 || dev >= kMaxDevices) return W4A16_EUNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W4A16_ECUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W4A16_ECUDA;
+    *addr = p;
     return W4A16_OK;
 }
 

@@ -1,35 +1,53 @@
-// gemm_tc.cu -- tcgen05 tensor-core W4A16 GEMM for sm_100a (the larger-M path).
+// gemm_tc.cu -- persistent stream-K tcgen05 tensor-core W4A16 GEMM for sm_100a (the larger-M path).
 //
 // C[M, N] = A[M, K] . dequant(W)[K, N], FP32 accumulation in tensor memory.
 // "4.3 Weight-only INT4", section 4: read, unpack, dequantize and multiply in one pipeline, each
 // weight byte crossing HBM once, data movement overlapped with on-chip compute; section 1: codes
-// dequantized on chip to FP16/BF16, multiply inputs stay 16-bit.
+// dequantized on chip to FP16/BF16, multiply inputs stay 16-bit. "INT8 vs INT4 Quantization, in
+// depth", "Two regimes": for tens of rows the layer still waits for memory, so every SM streams
+// weights; for hundreds it waits for the tensor cores.
 //
 // Mapping. The MMA computes D[n, m] = sum_k W^T[n, k] A^T[k, m] (swap-AB): the dequantized weight
-// tile (128 output channels x 64 K) is operand A (M_mma = 128), the activation tile
-// (BN rows of A x 64 K) is operand B (N_mma = BN), D (128 x BN, FP32) lives in tensor memory,
-// lane = output channel, column = row of A. One CTA computes one 128-channel x BN-row tile over
-// the whole K range.
+// tile (128 output channels x 64 K) is operand A (M_mma = 128), the activation tile (BN rows of
+// A x 64 K, 128-byte swizzle, loaded by TMA) is operand B (N_mma = BN), D (128 x BN, FP32) lives
+// in tensor memory, lane = output channel, column = row of A.
 //
-// Warp roles (192 threads):
-//   warp 0      : one thread issues, per 64-K stage, a TMA tile load of the activations
-//                 (128-byte swizzle), a bulk copy of the stage's 4 KiB of codes (half of a unit
-//                 record of the tiled buffer), and bulk copies of the stage's scales and zeros
-//                 from the same record.
-//   warp 1      : allocates tensor memory; one thread issues the four tcgen05.mma of a stage
-//                 and commits them to the stage's "empty" barrier.
-//   warps 2..5  : dequantize -- one thread per output channel turns its 64 codes of the stage
-//                 into 16-bit weights w = (u - z) * s (one rounding) and writes them into the
-//                 stage's A tile in the 128-byte-swizzled K-major layout; after the last stage
-//                 they read D back (tcgen05.ld) and store C.
-// Every wait on an mbarrier is bounded; on expiry the kernel records W4A16_ETIMEOUT in
-// dev_status and every role drains and returns, freeing its tensor memory.
+// Work split (stream-K). A tile is 128 output channels x one block of BN rows of A, the whole K;
+// tiles are ordered channel-major (the row blocks of one channel tile are neighbours, so their
+// weights are read from HBM once and from L2 after). The U = tiles x K/128 unit steps (one unit
+// record of the tiled buffer each) are cut into P contiguous ranges, one per SM, so every SM
+// streams the same number of weight bytes whatever the shape. A tile cut between CTAs cf < ... <
+// cl is the last of cf's range and the first of every later one: each later CTA publishes its
+// FP32 sums to the workspace and counts them (release, no wait); cf, after its own last unit,
+// waits for the count (acquire, bounded), adds the sums in CTA order, writes C and resets the
+// counter. The result does not depend on timing.
+//
+// Warp roles (512 threads):
+//   warp 0      : weight loader -- one bulk copy per two unit records (codes, scales and zeros
+//                 of 2 x 128 K, contiguous in the tiled buffer) into a ring of record slots.
+//   warp 1      : activation loader -- one TMA tile (BN rows x 64 K) per 64-K step into a ring;
+//                 owns the tensor memory allocation.
+//   warp 2      : MMA issuer -- one thread issues the four tcgen05.mma (K = 16 each) of a 64-K
+//                 step and commits them to the barriers that free the step's two operand slots;
+//                 after a tile's last step it commits the accumulator.
+//   warps 4..7  : epilogue -- tcgen05.ld of the accumulator (warp w reads lanes 32 (w % 4) ..),
+//                 then C (or the published partial sums of a cut tile); two accumulators in
+//                 tensor memory, so one tile's epilogue runs under the next tile's MMAs.
+//   warps 8..15 : dequantize -- thread (n, hh) turns the 32 codes of channel n in block
+//                 2 s + hh of a unit (s = 64-K half) into 16-bit weights (u - z) s (one rounding)
+//                 and writes them into the step's weight tile (128-byte-swizzled, K-major).
+// Record slots are freed by the dequant warps, activation and weight-tile slots by the MMA
+// commits, so the weight stream runs several units ahead of the tensor cores.
+// Every wait on an mbarrier or a tile counter is bounded; on expiry the kernel records
+// W4A16_ETIMEOUT in dev_status, every role stops, the loaders wait for their copies in flight,
+// the MMA thread waits for its last MMAs, and the CTA frees its tensor memory and returns.
 #include <cudaTypedefs.h>
 
 #include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
+#include "dequant.cuh"
 #include "sm100_ptx.cuh"
 #include "tiled_layout.cuh"
 
@@ -39,233 +57,394 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreadsTC = 320;  // producer, MMA, 8 dequant/epilogue warps
-constexpr uint64_t kSpin = 2000000000ull;  // a wait gives up after 2 s (nanoseconds)
+constexpr int kTcThreads = 512;
+constexpr int kTcWarpLoadW = 0, kTcWarpLoadA = 1, kTcWarpMma = 2, kTcWarpEpi = 4, kTcWarpDeq = 8;
+constexpr int kTcDeqWarps = 8;
+constexpr int kTcUnitsPerLoad = 2;     // unit records per record slot (one bulk copy)
+constexpr int kTcDTile = 128 * 128;    // weight tile of one 64-K step: 128 channels x 128 B
+constexpr int kTcSmemMax = 227 * 1024;
+constexpr int kTcMaxRing = 16;
+constexpr uint64_t kTcDrainNs = 2000000000ull;
 
-template <int BN>
-struct TcCfg {
-    static constexpr int kA = 128 * 128;           // dequantized weight tile: 128 rows x 128 B
-    static constexpr int kB = BN * 128;            // activation tile: BN rows x 128 B
-    static constexpr int kCodes = 4096;            // one tiled code tile
-    static constexpr int kScales = 2 * 256;        // up to two groups (group 32) x 128 fp16
-    static constexpr int kZeros = 2 * 64;          // up to two groups x 16 words
-    static constexpr int kStage = ((kA + kB + kCodes + kScales + kZeros + 1023) / 1024) * 1024;
-    static constexpr int kBudget = 227 * 1024 - 1024 - 256;  // alignment slack and barriers
-    static constexpr int kStagesRaw = kBudget / kStage;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-    static constexpr int kSmem = kStages * kStage + 1024 + 256;
-    static_assert(kStages >= 2, "pipeline needs two stages");
+struct TcParams {
+    const uint8_t* tiled;
+    void* C;
+    int* counters;      // one int per tile, zero between calls
+    float* partials;    // [P][BN][128]: sums a CTA publishes for the tile that opens its range
+    int* dev_status;
+    int M, K, N, sym, group;
+    uint32_t record, scales_off, zeros_off, slot_w;
+    int P, mblocks, nr, na, nd;
+    uint32_t off_a, off_w, off_bar;   // shared-memory offsets; the weight-tile ring starts at 0
+    uint64_t wait_ns;
+    GsMasks km;
 };
 
-template <typename T>
-struct Deq;
+__device__ __forceinline__ long long tc_unit_begin(int c, long long U, int P) { return ((long long)c * U) / P; }
+__device__ __forceinline__ int tc_unit_owner(long long u, long long U, int P) {
+    return (int)(((u + 1) * P - 1) / U);
+}
 
-// fp16: (1024 + u) - (1024 + z) is exact, one rounding in the product with s.
-template <>
-struct Deq<__half> {
-    static constexpr uint32_t kMagic = 0x64006400u;
-    __half2 zz, s2;
-    __device__ __forceinline__ void set(float s, int z) {
-        zz = __half2half2(__ushort_as_half((unsigned short)(0x6400 + z)));
-        s2 = __float2half2_rn(s);  // s is an fp16 value: exact
-    }
-    __device__ __forceinline__ uint32_t pair(uint32_t x) const {
-        __half2 h = *reinterpret_cast<__half2*>(&x);
-        __half2 r = __hmul2(__hsub2(h, zz), s2);
-        return *reinterpret_cast<uint32_t*>(&r);
-    }
-};
+__device__ __forceinline__ void tc_named_bar(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
-// bf16: d = (128 + u) - (128 + z) is exact; s = s_hi + s_lo with s_hi = s truncated to bf16 and
-// s_lo (at most 3 significant bits) exact in bf16; d * s_lo is exact, and
-// fma(d, s_hi, d * s_lo) rounds d * s once.
-template <>
-struct Deq<__nv_bfloat16> {
-    static constexpr uint32_t kMagic = 0x43004300u;
-    __nv_bfloat162 zz, shi, slo;
-    __device__ __forceinline__ void set(float s, int z) {
-        zz = __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)(0x4300 + z)));
-        const uint32_t sb = __float_as_uint(s) & 0xFFFF0000u;
-        const float hi = __uint_as_float(sb);
-        const float lo = s - hi;  // exact
-        shi = __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)(sb >> 16)));
-        slo = __float2bfloat162_rn(lo);  // exact
-    }
-    __device__ __forceinline__ uint32_t pair(uint32_t x) const {
-        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
-        __nv_bfloat162 d = __hsub2(h, zz);
-        __nv_bfloat162 t = __hmul2(d, slo);
-        __nv_bfloat162 r = __hfma2(d, shi, t);
-        return *reinterpret_cast<uint32_t*>(&r);
-    }
-};
+// Warp-uniform bounded wait.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status,
+                                        uint64_t ns) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, ns));
+}
+
+// Four K-consecutive MMAs D (+)= A . B^T (descriptors advanced by 32 bytes of K each), no commit.
+__device__ __forceinline__ void mma4_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %2, 0;\n\t"
+        "setp.eq.b32 t, %1, %1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %1, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %1, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %1, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %1, t;\n\t}" ::"r"(d_tmem),
+        "r"(idesc), "r"(accumulate), "l"(a_desc), "l"(b_desc), "l"(a_desc + 2), "l"(b_desc + 2), "l"(a_desc + 4),
+        "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
+        : "memory");
+}
 
 template <int BN, typename T>
-__global__ void __launch_bounds__(kThreadsTC, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restrict__ tiled, int M, int K,
-               int N, int group, int sym, const TiledLayout L, T* __restrict__ C, int* dev_status) {
-    using Cfg = TcCfg<BN>;
-    constexpr int NS = Cfg::kStages;
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
+    using Ops = GsOps<T>;
+    constexpr int kCols = BN < 32 ? 32 : BN;     // tensor-memory columns of one accumulator
+    constexpr uint32_t kSlotA = (uint32_t)BN * 128u;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * Cfg::kStage);
-    uint64_t* afull = full + NS;
-    uint64_t* empty = afull + NS;
-    uint64_t* accfull = empty + NS;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+    const int nr = p.nr, na = p.na, nd = p.nd;
+    uint8_t* ring_d = smem;
+    uint8_t* ring_a = smem + p.off_a;
+    uint8_t* ring_w = smem + p.off_w;
+    uint64_t* full_r = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+    uint64_t* empty_r = full_r + nr;
+    uint64_t* full_a = empty_r + nr;
+    uint64_t* empty_a = full_a + na;
+    uint64_t* full_d = empty_a + na;
+    uint64_t* empty_d = full_d + nd;
+    uint64_t* accfull = empty_d + nd;    // [2]
+    uint64_t* accempty = accfull + 2;    // [2]
+    uint64_t* lastmma = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lastmma + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nt = blockIdx.x;
-    const int n0 = nt * 128;
-    const int m0 = blockIdx.y * BN;
-    const int kstages = K / 64;
-    const int groups_per_stage = group >= 64 ? 1 : 64 / group;
+    const int UT = p.K / 128;                              // unit steps per tile
+    const long long tiles = (long long)(p.N / 128) * p.mblocks;
+    const long long U = tiles * UT;
+    const int cta = blockIdx.x, P = p.P;
+    const long long u0 = tc_unit_begin(cta, U, P), u1 = tc_unit_begin(cta + 1, U, P);
+    const uint32_t R = p.record;
+    const uint64_t wait_ns = p.wait_ns;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&afull[s], 256);
-            mbar_init(&empty[s], 1);
+        for (int i = 0; i < nr; ++i) {
+            mbar_init(&full_r[i], 1);
+            mbar_init(&empty_r[i], kTcDeqWarps);
         }
-        mbar_init(accfull, 1);
+        for (int i = 0; i < na; ++i) {
+            mbar_init(&full_a[i], 1);
+            mbar_init(&empty_a[i], 1);
+        }
+        for (int i = 0; i < nd; ++i) {
+            mbar_init(&full_d[i], kTcDeqWarps);
+            mbar_init(&empty_d[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], 4);
+        }
+        mbar_init(lastmma, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    if (warp == kTcWarpLoadA) {
+        tmem_alloc(tmem_slot, 2 * kCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_d = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ---------------------------------------------------------------- producer
+    if (warp == kTcWarpLoadW) {
+        // ------------------------------------------------------------ weight records
+        if (lane == 0) {
+            int rs = 0, issued[kTcMaxRing];
+            uint32_t rph = 0;
+            for (int i = 0; i < nr; ++i) issued[i] = 0;
+            for (long long i = u0; i < u1;) {
+                const long long tau = i / UT;
+                const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
+                const int n = (int)(seg_end - i < kTcUnitsPerLoad ? seg_end - i : kTcUnitsPerLoad);
+                if (!mbar_wait(&empty_r[rs], rph ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
+                const long long rec = (tau / p.mblocks) * UT + (i - tau * UT);
+                mbar_arrive_expect_tx(&full_r[rs], (uint32_t)n * R);
+                bulk_g2s(ring_w + (size_t)rs * p.slot_w, p.tiled + (size_t)rec * R, (uint32_t)n * R, &full_r[rs]);
+                ++issued[rs];
+                i += n;
+                if (++rs == nr) {
+                    rs = 0;
+                    rph ^= 1u;
+                }
+            }
+            // every copy issued lands before the CTA may exit
+            volatile int keep = 0;
+            for (int s = 0; s < nr; ++s)
+                if (issued[s] > 0) mbar_wait(&full_r[s], (uint32_t)(issued[s] - 1) & 1u, &keep, nullptr, kTcDrainNs);
+        }
+    } else if (warp == kTcWarpLoadA) {
+        // ------------------------------------------------------------ activation tiles
         if (lane == 0) {
             prefetch_tensormap(&tmA);
-            const uint32_t stage_bytes = (uint32_t)Cfg::kB + (uint32_t)Cfg::kCodes +
-                                         (uint32_t)groups_per_stage * (256u + (sym ? 0u : 64u));
-            int issued = 0;
-            for (int it = 0; it < kstages; ++it) {
-                const int s = it % NS;
-                const uint32_t r = (uint32_t)(it / NS);
-                if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, dev_status, kSpin)) break;
-                uint8_t* st = smem + s * Cfg::kStage;
-                mbar_arrive_expect_tx(&full[s], stage_bytes);
-                tma_2d_g2s(st + Cfg::kA, &tmA, it * 64, m0, &full[s]);
-                // unit record (nt, it / 2): blocks 2 (it % 2), 2 (it % 2) + 1 of its codes, and
-                // the record's groups that fall in this stage (contiguous in the record)
-                const uint8_t* rec = tiled + ((size_t)nt * (K / 128) + it / 2) * L.record;
-                bulk_g2s(st + Cfg::kA + Cfg::kB, rec + (it & 1) * 4096, 4096, &full[s]);
-                const int lg0 = (it * 64) / group - (it / 2) * L.groups;
-                bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes, rec + L.scales + lg0 * 256, groups_per_stage * 256,
-                         &full[s]);
-                if (!sym)
-                    bulk_g2s(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales, rec + L.zeros + lg0 * 64,
-                             groups_per_stage * 64, &full[s]);
-                ++issued;
-            }
-            // drain: every copy issued has landed before the block may exit
-            for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it) {
-                const int s = it % NS;
-                mbar_wait(&full[s], (uint32_t)(it / NS) & 1u, abort_flag, dev_status, kSpin);
-            }
-        }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(BN, sizeof(T) == 2 && !std::is_same<T, __half>::value);
-            int done = 0;
-            for (int it = 0; it < kstages; ++it) {
-                const int s = it % NS;
-                const uint32_t r = (uint32_t)(it / NS);
-                if (!mbar_wait(&full[s], r & 1u, abort_flag, dev_status, kSpin)) break;
-                if (!mbar_wait(&afull[s], r & 1u, abort_flag, dev_status, kSpin)) break;
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + s * Cfg::kStage);
-                const uint32_t b_base = a_base + Cfg::kA;
-                // the stage's four K-steps of 16 and the commit that frees the stage
-                mma4_f16_ss_commit(tmem_d, smem_desc_sw128(a_base), smem_desc_sw128(b_base), idesc,
-                                   it > 0 ? 1u : 0u, &empty[s]);
-                ++done;
-            }
-            mma_commit(accfull);  // also completes when nothing was issued
-            (void)done;
-        }
-    } else {
-        // ---------------------------------------------------------------- dequant + epilogue
-        // two warps per TMEM lane quarter: warp half hf dequantizes rows 4 hf .. 4 hf + 3 of the
-        // stage's code tile (K 32 hf .. 32 hf + 31) and stores columns [BN/2 hf, BN/2 (hf + 1)) of C
-        const int q = warp & 3;           // tensor-memory lane quarter this warp may access
-        const int hf = (warp - 2) >> 2;   // 0 for warps 2..5, 1 for warps 6..9
-        const int n = 32 * q + lane;      // output channel within the tile = TMEM lane
-        Deq<T> dq;
-        bool ok = true;
-        for (int it = 0; it < kstages && ok; ++it) {
-            const int s = it % NS;
-            const uint32_t r = (uint32_t)(it / NS);
-            ok = mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, dev_status, kSpin) &&
-                 mbar_wait(&full[s], r & 1u, abort_flag, dev_status, kSpin);
-            if (!ok) break;
-            uint8_t* st = smem + s * Cfg::kStage;
-            const uint4* ctile = reinterpret_cast<const uint4*>(st + Cfg::kA + Cfg::kB);
-            const __half* ssm = reinterpret_cast<const __half*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes);
-            const uint32_t* zsm = reinterpret_cast<const uint32_t*>(st + Cfg::kA + Cfg::kB + Cfg::kCodes + Cfg::kScales);
-            uint8_t* atile = st;
-            // rows 4 hf .. 4 hf + 3 of the stage: block h = 2 (it % 2) + hf of the unit record,
-            // channel n in slot n ^ 2h
-            const uint4 w4 = ctile[128 * hf + (n ^ (2 * (2 * (it & 1) + hf)))];
-            const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
-            // group of this half inside the stage (group 32: one group per half)
-            const int lg = groups_per_stage > 1 ? hf : 0;
-            const float sv = __half2float(ssm[lg * 128 + n]);
-            const int zv = sym ? 8 : (int)((zsm[lg * 16 + n / 8] >> (4 * (n % 8))) & 0xFu);
-            dq.set(sv, zv);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int jl = 4 * hf + i;
-                const uint32_t w = words[i];
-                uint4 out;
-                out.x = dq.pair((w & 0x000F000Fu) | Deq<T>::kMagic);
-                out.y = dq.pair(((w >> 4) & 0x000F000Fu) | Deq<T>::kMagic);
-                out.z = dq.pair(((w >> 8) & 0x000F000Fu) | Deq<T>::kMagic);
-                out.w = dq.pair(((w >> 12) & 0x000F000Fu) | Deq<T>::kMagic);
-                const int row = n;
-                const uint32_t off = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((jl ^ (row & 7)) << 4));
-                *reinterpret_cast<uint4*>(atile + off) = out;
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&afull[s]);
-        }
-        // epilogue: D (lane n, columns 0..BN-1) -> C[m0 + m, n0 + n]; this warp stores half the columns
-        if (mbar_wait(accfull, 0, abort_flag, dev_status, kSpin) && ok && !*abort_flag) {
-            tc_fence_after();
-            const uint32_t lane_base = tmem_d + ((uint32_t)(32 * q) << 16);
-            constexpr int kChunks = BN / 16;
-            const int c0 = kChunks > 1 ? hf * (kChunks / 2) : 0;
-            const int c1 = kChunks > 1 ? c0 + kChunks / 2 : (hf == 0 ? 1 : 0);
-#pragma unroll 1
-            for (int c = c0; c < c1; ++c) {
-                uint32_t v[16];
-                tmem_ld16(lane_base + c * 16, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int m = m0 + c * 16 + i;
-                    if (m < M) C[(size_t)m * N + n0 + n] = Act<T>::from_f32(__uint_as_float(v[i]));
+            int as = 0, issued[kTcMaxRing];
+            uint32_t aph = 0;
+            bool ok = true;
+            for (int i = 0; i < na; ++i) issued[i] = 0;
+            for (long long i = u0; i < u1 && ok; ++i) {
+                const long long tau = i / UT;
+                const int mb = (int)(tau % p.mblocks);
+                const int ku = (int)(i - tau * UT);
+                for (int h = 0; h < 2; ++h) {
+                    if (!mbar_wait(&empty_a[as], aph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full_a[as], kSlotA);
+                    tma_2d_g2s(ring_a + (size_t)as * kSlotA, &tmA, ku * 128 + h * 64, mb * BN, &full_a[as]);
+                    ++issued[as];
+                    if (++as == na) {
+                        as = 0;
+                        aph ^= 1u;
+                    }
                 }
+            }
+            volatile int keep = 0;
+            for (int s = 0; s < na; ++s)
+                if (issued[s] > 0) mbar_wait(&full_a[s], (uint32_t)(issued[s] - 1) & 1u, &keep, nullptr, kTcDrainNs);
+        }
+    } else if (warp == kTcWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16(BN, std::is_same<T, __nv_bfloat16>::value);
+            int as = 0, ds = 0, use[2] = {0, 0}, ab = 0;
+            uint32_t aph = 0, dph = 0;
+            bool ok = true;
+            for (long long i = u0; i < u1 && ok;) {
+                const long long tau = i / UT;
+                const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
+                if (!mbar_wait(&accempty[ab], ((uint32_t)use[ab] & 1u) ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(ab * kCols);
+                bool first = true;
+                for (; i < seg_end && ok; ++i) {
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait(&full_d[ds], dph, abort_flag, p.dev_status, wait_ns) ||
+                            !mbar_wait(&full_a[as], aph, abort_flag, p.dev_status, wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        mma4_f16_ss(d_tmem, smem_desc_sw128(smem_u32(ring_d + (size_t)ds * kTcDTile)),
+                                    smem_desc_sw128(smem_u32(ring_a + (size_t)as * kSlotA)), idesc, first ? 0u : 1u);
+                        mma_commit(&empty_a[as]);
+                        mma_commit(&empty_d[ds]);
+                        first = false;
+                        if (++as == na) {
+                            as = 0;
+                            aph ^= 1u;
+                        }
+                        if (++ds == nd) {
+                            ds = 0;
+                            dph ^= 1u;
+                        }
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&accfull[ab]);
+                ++use[ab];
+                ab ^= 1;
+            }
+            // the CTA exits only after its last MMAs completed
+            mma_commit(lastmma);
+            volatile int keep = 0;
+            mbar_wait(lastmma, 0, &keep, nullptr, kTcDrainNs);
+        }
+    } else if (warp >= kTcWarpEpi && warp < kTcWarpEpi + 4) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                   // tensor-memory lane quarter
+        const int n = 32 * q + lane;              // channel within the tile
+        const bool leader = warp == kTcWarpEpi && lane == 0;
+        T* C = static_cast<T*>(p.C);
+        int use[2] = {0, 0}, ab = 0;
+        bool ok = true;
+        for (long long i = u0; i < u1;) {
+            const long long tau = i / UT;
+            const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
+            i = seg_end;
+            ok = ok && tc_wait(&accfull[ab], (uint32_t)use[ab] & 1u, abort_flag, p.dev_status, wait_ns);
+            tc_fence_after();
+            const int nt = (int)(tau / p.mblocks), mb = (int)(tau % p.mblocks);
+            const size_t n0 = (size_t)nt * 128;
+            const int m0 = mb * BN;
+            const int cf = tc_unit_owner(tau * UT, U, P), cl = tc_unit_owner(tau * UT + UT - 1, U, P);
+            const uint32_t lane_base = tmem + (uint32_t)(ab * kCols) + ((uint32_t)(32 * q) << 16);
+            if (cf == cl || cta == cf) {
+                if (cf != cl) {
+                    // the tile is cut between CTAs cf .. cl and this is cf: wait until every later
+                    // CTA of the tile has published its sums (the tile opens their ranges)
+                    if (leader) {
+                        const uint64_t t0 = globaltimer_ns();
+                        for (;;) {
+                            int c;
+                            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(c) : "l"(p.counters + tau)
+                                         : "memory");
+                            if (c >= cl - cf) break;
+                            if (*abort_flag || globaltimer_ns() - t0 > wait_ns) {
+                                *abort_flag = 1;
+                                report_status(p.dev_status, W4A16_ETIMEOUT);
+                                break;
+                            }
+                        }
+                        p.counters[tau] = 0;
+                    }
+                    tc_named_bar(1, 128);
+                }
+                if (ok && !*abort_flag) {
+#pragma unroll 1
+                    for (int c = 0; c < BN / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(lane_base + (uint32_t)(c * 16), v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int mr = c * 16 + j, m = m0 + mr;
+                            if (m < p.M) {
+                                float y = __uint_as_float(v[j]);
+                                for (int cc = cf + 1; cc <= cl; ++cc)
+                                    y += __ldcg(p.partials + ((size_t)cc * BN + mr) * 128 + n);
+                                C[(size_t)m * p.N + n0 + n] = Act<T>::from_f32(y);
+                            }
+                        }
+                    }
+                }
+            } else {
+                // a later CTA of a cut tile (the tile opens its range): publish the sums and count
+                // them, without waiting
+                if (ok && !*abort_flag) {
+                    float* part = p.partials + (size_t)cta * BN * 128;
+#pragma unroll 1
+                    for (int c = 0; c < BN / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(lane_base + (uint32_t)(c * 16), v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int mr = c * 16 + j;
+                            if (m0 + mr < p.M) __stcg(part + (size_t)mr * 128 + n, __uint_as_float(v[j]));
+                        }
+                    }
+                }
+                __threadfence();
+                tc_named_bar(1, 128);
+                if (leader) asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + tau) : "memory");
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[ab]);
+            ++use[ab];
+            ab ^= 1;
+        }
+    } else if (warp >= kTcWarpDeq) {
+        // ------------------------------------------------------------ dequantize
+        const int dt = threadIdx.x - 32 * kTcWarpDeq;
+        const int n = dt & 127, hh = dt >> 7;
+        const int sym = p.sym, group = p.group;
+        const GsMasks km = p.km;
+        const uint32_t swz = (uint32_t)(n & 7);
+        const uint32_t row_off = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
+        int rs = 0, ds = 0;
+        uint32_t rph = 0, dph = 0;
+        bool ok = true;
+        for (long long i = u0; i < u1 && ok;) {
+            const long long tau = i / UT;
+            const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
+            const int nu = (int)(seg_end - i < kTcUnitsPerLoad ? seg_end - i : kTcUnitsPerLoad);
+            i += nu;
+            if (!tc_wait(&full_r[rs], rph, abort_flag, p.dev_status, wait_ns)) {
+                ok = false;
+                break;
+            }
+            for (int uu = 0; uu < nu && ok; ++uu) {
+                const uint8_t* rec = ring_w + (size_t)rs * p.slot_w + (size_t)uu * R;
+                // this thread's 32-K blocks of the unit's two 64-K halves, with their scale and zero
+                uint4 cw[2];
+                uint16_t sb[2];
+                uint32_t zv[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int blk = 2 * h + hh;
+                    cw[h] = *reinterpret_cast<const uint4*>(rec + 2048 * blk + 16 * (n ^ (2 * blk)));
+                    const int lg = (32 * blk) / group;
+                    sb[h] = *reinterpret_cast<const uint16_t*>(rec + p.scales_off + 256 * lg + 2 * n);
+                    zv[h] = sym ? 8u
+                                : (*reinterpret_cast<const uint32_t*>(rec + p.zeros_off + 64 * lg + 4 * (n >> 3)) >>
+                                   (4 * (n & 7))) & 0xFu;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (!tc_wait(&empty_d[ds], dph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t za = Ops::zz_a(zv[h]), zb = Ops::zz_b(zv[h]);
+                    typename Ops::Scale sc;
+                    sc.set(sb[h]);
+                    uint8_t* tile = ring_d + (size_t)ds * kTcDTile;
+                    const uint32_t words[4] = {cw[h].x, cw[h].y, cw[h].z, cw[h].w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t r[4];
+                        Ops::unpack(words[w], km, r);
+                        uint4 out;
+                        out.x = sc.apply(Ops::sub_a(r[0], za));
+                        out.y = sc.apply(Ops::sub_b(r[1], zb));
+                        out.z = sc.apply(Ops::sub_a(r[2], za));
+                        out.w = sc.apply(Ops::sub_b(r[3], zb));
+                        const uint32_t j = (uint32_t)(4 * hh + w);   // 16-byte chunk (8 K) of the 64-K row
+                        *reinterpret_cast<uint4*>(tile + row_off + ((j ^ swz) << 4)) = out;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_d[ds]);
+                    if (++ds == nd) {
+                        ds = 0;
+                        dph ^= 1u;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_r[rs]);
+            if (++rs == nr) {
+                rs = 0;
+                rph ^= 1u;
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kTcWarpLoadA) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, Cfg::kTmemCols);
+        tmem_dealloc(tmem, 2 * kCols);
     }
 }
 
@@ -276,16 +455,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(q);
     });
     return fn;
 }
 
-// Activations A [M, K] (16-bit, row-major) as a 2-D tensor map: box 64 (K) x BN (rows),
+// Activations A [M, K] (16-bit, row-major) as a 2-D tensor map: box 64 (K) x box_rows,
 // 128-byte swizzle; rows past M read as zero.
 bool make_act_map(CUtensorMap* map, const void* A, int M, int K, int box_rows, bool bf16) {
     auto fn = encode_fn();
@@ -316,45 +495,115 @@ bool make_u8_map(CUtensorMap* map, const void* base, int rows, int K, int box_ro
     return r == CUDA_SUCCESS;
 }
 
+int tc_block_rows(int M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
+    TcPlan pl = {};
+    if (M < 1 || K % 128 != 0 || N % 128 != 0 || K < 128 || N < 128 || n_sm <= 0) return pl;
+    const TiledLayout L = tiled_layout(K, N, group, sym);
+    pl.bn = tc_block_rows(M);
+    pl.mblocks = (M + pl.bn - 1) / pl.bn;
+    const long long tiles = (long long)(N / 128) * pl.mblocks;
+    if (tiles > kGemvStreamMaxTiles) return pl;
+    const long long units = tiles * (K / 128);
+    pl.ctas = (int)(units < n_sm ? units : n_sm);
+    pl.slot_w = (uint32_t)((kTcUnitsPerLoad * L.record + 127) & ~127u);
+    const uint32_t slot_a = (uint32_t)pl.bn * 128u;
+    pl.nd = 3;
+    pl.na = pl.bn >= 256 ? 3 : 4;
+    const size_t bars = 1024;   // barriers, tensor-memory slot, abort flag
+    const size_t fixed = 1024 /* alignment */ + (size_t)pl.nd * kTcDTile + (size_t)pl.na * slot_a + bars;
+    if (fixed >= (size_t)kTcSmemMax) return TcPlan{};
+    size_t nr = ((size_t)kTcSmemMax - fixed) / pl.slot_w;
+    if (nr > kTcMaxRing) nr = kTcMaxRing;
+    if (nr < 2) return TcPlan{};
+    pl.nr = (int)nr;
+    pl.off_a = (uint32_t)pl.nd * kTcDTile;
+    pl.off_w = pl.off_a + (uint32_t)pl.na * slot_a;
+    pl.off_bar = pl.off_w + (uint32_t)pl.nr * pl.slot_w;
+    pl.off_bar = (pl.off_bar + 127u) & ~127u;
+    pl.smem = 1024 + pl.off_bar + bars;
+    pl.partial_bytes = (size_t)pl.ctas * pl.bn * 128 * sizeof(float);
+    pl.ok = pl.smem <= (size_t)kTcSmemMax;
+    return pl;
+}
+
 namespace {
 
 template <int BN, typename T>
-int launch_tc_typed(const void* A, int M, int K, const void* tiled, int N, int group, int sym, void* C,
-                    int* dev_status, cudaStream_t stream) {
-    using Cfg = TcCfg<BN>;
+int launch_tc_typed(const CUtensorMap& map, const TcParams& prm, size_t smem, cudaStream_t stream) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
         attr_err = cudaFuncSetAttribute(tc_gemm_kernel<BN, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        Cfg::kSmem);
+                                        kTcSmemMax);
     });
     if (attr_err != cudaSuccess) return W4A16_ECUDA;
-    CUtensorMap map;
-    if (!make_act_map(&map, A, M, K, BN, !std::is_same<T, __half>::value)) return W4A16_ECUDA;
-    const TiledLayout L = tiled_layout(K, N, group, sym);
-    dim3 grid(N / 128, (M + BN - 1) / BN);
-    tc_gemm_kernel<BN, T><<<grid, kThreadsTC, Cfg::kSmem, stream>>>(
-        map, static_cast<const uint8_t*>(tiled), M, K, N, group, sym, L, static_cast<T*>(C), dev_status);
+    tc_gemm_kernel<BN, T><<<prm.P, kTcThreads, smem, stream>>>(map, prm);
     return launch_status();
 }
 
 template <typename T>
-int launch_tc_bn(const void* A, int M, int K, const void* tiled, int N, int group, int sym, void* C,
-                 int* dev_status, cudaStream_t stream) {
-    if (M <= 16) return launch_tc_typed<16, T>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
-    if (M <= 32) return launch_tc_typed<32, T>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
-    if (M <= 64) return launch_tc_typed<64, T>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
-    if (M <= 128) return launch_tc_typed<128, T>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
-    return launch_tc_typed<256, T>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
+int launch_tc_bn(int bn, const CUtensorMap& map, const TcParams& prm, size_t smem, cudaStream_t stream) {
+    switch (bn) {
+        case 16: return launch_tc_typed<16, T>(map, prm, smem, stream);
+        case 32: return launch_tc_typed<32, T>(map, prm, smem, stream);
+        case 64: return launch_tc_typed<64, T>(map, prm, smem, stream);
+        case 128: return launch_tc_typed<128, T>(map, prm, smem, stream);
+        case 256: return launch_tc_typed<256, T>(map, prm, smem, stream);
+        default: return W4A16_EUNSUPPORTED;
+    }
 }
 
 }  // namespace
 
 int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, int N, int group, int sym,
-                   void* C, int* dev_status, cudaStream_t stream) {
-    if (a_dtype == W4A16_BF16)
-        return launch_tc_bn<__nv_bfloat16>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
-    return launch_tc_bn<__half>(A, M, K, tiled, N, group, sym, C, dev_status, stream);
+                   void* C, void* workspace, int* dev_status, cudaStream_t stream) {
+    const TcPlan pl = plan_gemm_tc(M, N, K, group, sym, gemv_stream_sm_count());
+    if (!pl.ok) return W4A16_EUNSUPPORTED;
+    if (!workspace) return W4A16_EWORKSPACE;
+    const bool bf16 = a_dtype == W4A16_BF16;
+    CUtensorMap map;
+    if (!make_act_map(&map, A, M, K, pl.bn, bf16)) return W4A16_ECUDA;
+    const TiledLayout L = tiled_layout(K, N, group, sym);
+    TcParams prm = {};
+    prm.tiled = static_cast<const uint8_t*>(tiled);
+    prm.C = C;
+    prm.counters = static_cast<int*>(workspace);
+    prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kGemvStreamCounterBytes);
+    prm.dev_status = dev_status;
+    prm.M = M;
+    prm.K = K;
+    prm.N = N;
+    prm.sym = sym;
+    prm.group = group;
+    prm.record = L.record;
+    prm.scales_off = L.scales;
+    prm.zeros_off = L.zeros;
+    prm.slot_w = pl.slot_w;
+    prm.P = pl.ctas;
+    prm.mblocks = pl.mblocks;
+    prm.nr = pl.nr;
+    prm.na = pl.na;
+    prm.nd = pl.nd;
+    prm.off_a = pl.off_a;
+    prm.off_w = pl.off_w;
+    prm.off_bar = pl.off_bar;
+    prm.wait_ns = wait_limit_ns();
+    prm.km.lo = 0x000F000Fu;
+    prm.km.hi = bf16 ? 0x000F000Fu : 0x00F000F0u;
+    prm.km.magic = bf16 ? 0x43004300u : 0x64006400u;
+    prm.km.m4 = 1u << 28;
+    prm.km.m8 = 1u << 24;
+    prm.km.m12 = 1u << 20;
+    if (bf16) return launch_tc_bn<__nv_bfloat16>(pl.bn, map, prm, pl.smem, stream);
+    return launch_tc_bn<__half>(pl.bn, map, prm, pl.smem, stream);
 }
 
 }  // namespace w4a16

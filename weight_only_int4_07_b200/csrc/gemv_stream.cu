@@ -38,6 +38,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "dequant.cuh"
 #include "sm100_ptx.cuh"
 #include "tiled_layout.cuh"
 
@@ -54,114 +55,6 @@ constexpr int kGsSmemMax = 227 * 1024;
 constexpr uint64_t kGsSpin = 2000000000ull;
 constexpr int kGsZrowBytes = 512;   // the zero activation block, then per-row exponent bounds
 
-__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {   // a >> k for b = 2^(32-k)
-    uint32_t r;
-    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t andor(uint32_t a, uint32_t b, uint32_t c) {   // (a & b) | c
-    uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-
-// Masks and shift multipliers, passed at run time so that the compiler keeps them in registers:
-// one lop3 per operand register, shifts on the multiply pipe.
-struct GsMasks {
-    uint32_t lo, hi, magic, m4, m8, m12;
-};
-
-template <typename T>
-struct GsOps;
-
-template <>
-struct GsOps<__half> {
-    // operands: r0 = elements (0,1), r2 = (4,5) as 1024 + u; r1 = (2,3), r3 = (6,7) as 1024 + 16 u
-    static __device__ __forceinline__ void unpack(uint32_t w, const GsMasks& k, uint32_t (&r)[4]) {
-        const uint32_t h = mulhi(w, k.m8);
-        r[0] = andor(w, k.lo, k.magic);
-        r[1] = andor(w, k.hi, k.magic);
-        r[2] = andor(h, k.lo, k.magic);
-        r[3] = andor(h, k.hi, k.magic);
-    }
-    static __device__ __forceinline__ uint32_t zz_a(uint32_t z) { return (0x6400u + z) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t zz_b(uint32_t z) { return (0xD400u + (z << 4)) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {   // (1024+u) - (1024+z)
-        uint32_t r;
-        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(zz));
-        return r;
-    }
-    static __device__ __forceinline__ uint32_t sub_b(uint32_t x, uint32_t zz) {   // x / 16 - (64 + z)
-        uint32_t r;
-        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(0x2C002C00u), "r"(zz));
-        return r;
-    }
-    struct Scale {   // d * s, one rounding (s is an fp16 value)
-        uint32_t s2;
-        __device__ __forceinline__ void set(uint16_t bits) { s2 = (uint32_t)bits * 0x00010001u; }
-        __device__ __forceinline__ uint32_t apply(uint32_t d) const {
-            uint32_t r;
-            asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(d), "r"(s2));
-            return r;
-        }
-    };
-    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-            "{%0, %1, %2, %3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-};
-
-template <>
-struct GsOps<__nv_bfloat16> {
-    // operands: all four registers as 128 + u (elements (0,1), (2,3), (4,5), (6,7))
-    static __device__ __forceinline__ void unpack(uint32_t w, const GsMasks& k, uint32_t (&r)[4]) {
-        r[0] = andor(w, k.lo, k.magic);
-        r[1] = andor(mulhi(w, k.m4), k.lo, k.magic);
-        r[2] = andor(mulhi(w, k.m8), k.lo, k.magic);
-        r[3] = andor(mulhi(w, k.m12), k.lo, k.magic);
-    }
-    static __device__ __forceinline__ uint32_t zz_a(uint32_t z) { return (0x4300u + z) * 0x00010001u; }
-    static __device__ __forceinline__ uint32_t zz_b(uint32_t z) { return zz_a(z); }
-    static __device__ __forceinline__ uint32_t sub_a(uint32_t x, uint32_t zz) {   // (128+u) - (128+z)
-        uint32_t r;
-        asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(zz));
-        return r;
-    }
-    static __device__ __forceinline__ uint32_t sub_b(uint32_t x, uint32_t zz) { return sub_a(x, zz); }
-    struct Scale {   // d * s rounded once: s = s_hi (bf16 truncation of s) + s_lo (exact in bf16)
-        uint32_t hi2, lo2;
-        __device__ __forceinline__ void set(uint16_t bits) {
-            const float s = __half2float(__ushort_as_half(bits));
-            const uint32_t sb = __float_as_uint(s) & 0xFFFF0000u;
-            hi2 = (sb >> 16) * 0x00010001u;
-            __nv_bfloat162 l = __float2bfloat162_rn(s - __uint_as_float(sb));
-            lo2 = *reinterpret_cast<uint32_t*>(&l);
-        }
-        __device__ __forceinline__ uint32_t apply(uint32_t d) const {
-            uint32_t t, r;
-            asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(d), "r"(lo2));
-            asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(d), "r"(hi2), "r"(t));
-            return r;
-        }
-    };
-    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-            "{%0, %1, %2, %3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-};
-
-template <typename X>
-struct OpsTag {
-    using type = X;
-};
-
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -173,9 +66,10 @@ __device__ __forceinline__ long long unit_begin(int c, long long U, int P) { ret
 __device__ __forceinline__ int unit_owner(long long u, long long U, int P) { return (int)(((u + 1) * P - 1) / U); }
 
 // Warp-uniform bounded wait: the common case (phase already complete) costs one try and a vote.
-__device__ __forceinline__ bool wait_uniform(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status) {
+__device__ __forceinline__ bool wait_uniform(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status,
+                                             uint64_t limit_ns) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, kGsSpin));
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, limit_ns));
 }
 
 struct GsParams {
@@ -195,6 +89,7 @@ struct GsParams {
     // out_f32 set the FP32 sums go there ([M][N]) instead of C
     int lda, c0, ktot;
     float* out_f32;
+    uint64_t wait_ns;   // limit of every bounded wait (the drain after a timeout keeps kGsSpin)
 };
 
 // NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
@@ -431,7 +326,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                             asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + tile)
                                          : "memory");
                             if (n >= cl - cf) break;
-                            if (*abort_flag || globaltimer_ns() - t0 > kGsSpin) {
+                            if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
                                 *abort_flag = 1;
                                 report_status(p.dev_status, W4A16_ETIMEOUT);
                                 break;
@@ -598,7 +493,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
             s_idx = 0;
             ph ^= 1u;
         }
-        if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status)) aborted = true;
+        if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status, p.wait_ns)) aborted = true;
         const int li = st * kGsUnitsPerStage + grp;
         if (li >= nunits) continue;
         while (li >= seg_hi) emit();
@@ -782,6 +677,7 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.red_bytes = (uint32_t)pl.red_bytes;
     prm.lda = K;
     prm.ktot = K / 128;
+    prm.wait_ns = wait_limit_ns();
     const bool bf16 = a_dtype == W4A16_BF16;
     const bool bf16_math = bf16 && group != 128;   // bf16 at group 128 runs the fp16 arithmetic
     prm.km.lo = 0x000F000Fu;

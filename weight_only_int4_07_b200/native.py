@@ -84,6 +84,8 @@ def lib():
     L.w4a16_status_str.restype = ctypes.c_char_p
     L.w4a16_version.argtypes = []
     L.w4a16_version.restype = I
+    L.w4a16_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.w4a16_set_wait_limit_ns.restype = ctypes.c_uint64
     _lib = L
     return L
 
@@ -110,6 +112,12 @@ w4a16_status_str = status_str
 
 def w4a16_version() -> int:
     return int(lib().w4a16_version())
+
+
+def w4a16_set_wait_limit_ns(ns: int) -> int:
+    """Limit of every bounded device wait for later launches (0 = the 2 s default); returns the
+    previous limit."""
+    return int(lib().w4a16_set_wait_limit_ns(int(ns)))
 
 
 def w4a16_quantize(W, group, sym, codes=None, scales=None, zeros=None, dev_status=None):
