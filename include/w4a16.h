@@ -311,6 +311,13 @@ W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
  *   dev_status device int or NULL: set to W4A16_ETIMEOUT if a bounded on-device wait gave up
  *              (the output is then unspecified; the device stays usable).
  *   stream     cudaStream_t.
+ * Ordering. The decode kernel (tiled layout, M <= 16) is launched with programmatic dependent
+ * launch: it may start while the kernel before it on the stream is still running, and it
+ * starts streaming the tiled weight buffer before it waits for that kernel (it waits before it
+ * reads A). The weight buffer must therefore not be written by the kernel that immediately
+ * precedes w4a16_gemm on the stream, unless that kernel makes its writes visible device-wide
+ * before its threads exit, as w4a16_repack does; a memory copy, an event or any other stream
+ * operation in between also orders them. A, C and the workspace carry no such condition.
  * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
  * W4A16_ECUDA.
  */

@@ -1,12 +1,16 @@
 """The bounded device waits run out on purpose, and the device stays usable.
 
 Every wait inside the kernels (a pipeline barrier, or a tile counter that another CTA of the
-same launch sets) gives up after a time limit. w4a16_set_wait_limit_ns(1) shortens that limit to
-1 ns, so the first wait that is not already satisfied gives up: the kernel records W4A16_ETIMEOUT
-in dev_status, stops issuing, lets its copies and MMAs in flight complete, frees its tensor memory
-and returns. Nothing here faults, traps or spins without a limit. The test then restores the
-default limit, zeroes the workspace again (the header asks for that after a timeout) and checks
-that the next call on the same device is exact against the oracle.
+same launch sets) gives up after a time limit, and each suspension of a waiting thread is at most
+that limit. Two ways to make the waits run out, neither of which faults or traps anything:
+  * w4a16_set_wait_limit_ns(1): the first pipeline wait whose copy has not landed within 1 ns
+    gives up, in the middle of the weight stream, with copies and MMAs in flight;
+  * tile counters that start far below zero instead of at zero (a flag nothing will set): the
+    CTA that sums a cut tile waits for a count it never sees (limit 1 ms).
+Either way the kernel records W4A16_ETIMEOUT in dev_status, stops issuing, lets its copies and
+MMAs in flight complete, frees its tensor memory and returns. The test then restores the default
+limit, zeroes the workspace again (the header asks for that after a timeout) and checks that the
+next call on the same device is exact against the oracle.
 """
 import numpy as np
 import pytest
@@ -41,17 +45,20 @@ def _layer(K, N, group, sym, seed):
     return (oc, os_, oz), native.w4a16_repack(gc, gs, gz, K, N, group, sym)
 
 
+@pytest.mark.parametrize("how", ["limit", "counters"])
 @pytest.mark.parametrize("M,kernel", [(1, native.KERNEL_GEMV), (8, native.KERNEL_GEMV),
                                       (64, native.KERNEL_TC), (256, native.KERNEL_TC)])
-def test_waits_run_out_then_the_device_recovers(M, kernel):
+def test_waits_run_out_then_the_device_recovers(M, kernel, how):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     (oc, os_, oz), tiled = _layer(K, N, group, sym, 21)
     Ab = synthetic.activations(M, K, 22 + M, dtype=a_dtype)
     A = torch.from_numpy(Ab.view(np.int16)).view(torch.bfloat16).cuda()
     ws = torch.zeros(native.w4a16_workspace_bytes(M, N, K, group), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if how == "counters":
+        ws[:65536] = 0x80                   # every tile counter reads as -2139062144
     torch.cuda.synchronize()
-    prev = native.w4a16_set_wait_limit_ns(1)
+    prev = native.w4a16_set_wait_limit_ns(1 if how == "limit" else 1_000_000)
     try:
         native.w4a16_gemm(A, tiled, None, None, N, group, sym, layout=native.LAYOUT_TILED, kernel=kernel,
                           workspace=ws, dev_status=status)

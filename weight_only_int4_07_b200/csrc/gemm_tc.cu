@@ -92,7 +92,7 @@ __device__ __forceinline__ void tc_named_bar(int id, int threads) {
 // Warp-uniform bounded wait.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status,
                                         uint64_t ns) {
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, ns));
 }
 

@@ -180,8 +180,10 @@ GemvPlan plan_gemv_plain(int M, int N, int K, int group) {
     const int rows = K / 8;
     const int rows_per_group = group / 8;
     const int blocks_x = (N / 4 + kThreads - 1) / kThreads;
-    // aim for about four blocks per SM of a 148-SM B200
-    const int target_blocks = 4 * 148;
+    // aim for about four blocks per SM (148 SMs when no device answers, as on a build host)
+    int n_sm = gemv_stream_sm_count();
+    if (n_sm <= 0) n_sm = 148;
+    const int target_blocks = 4 * n_sm;
     int splits = (target_blocks + blocks_x - 1) / blocks_x;
     splits = splits < 1 ? 1 : splits;
     int rps = (rows + splits - 1) / splits;

@@ -68,7 +68,7 @@ __device__ __forceinline__ int unit_owner(long long u, long long U, int P) { ret
 // Warp-uniform bounded wait: the common case (phase already complete) costs one try and a vote.
 __device__ __forceinline__ bool wait_uniform(uint64_t* bar, uint32_t parity, volatile int* abort, int* dev_status,
                                              uint64_t limit_ns) {
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, limit_ns));
 }
 
@@ -469,6 +469,89 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         }
     };
 
+    // Group 128 on the fp16 arithmetic: the codes enter the MMAs as fp16 subnormals, u 2^-24 for
+    // the pairs (0, 1) and (4, 5) of a word and 16 u 2^-24 for (2, 3) and (6, 7), each operand
+    // register one AND of the word (no magic, no zero-point arithmetic), summed in two chains
+    // (lo, hi) per row tile. The zero point comes off after the MMAs: per unit the same two chains
+    // run on constant operands whose row j holds j 2^-24 (16 j 2^-24), which gives
+    // sum_k a_k j 2^-24 for every zero j = 0..15, and each channel takes the row of its own zero
+    // (a shuffle from the lane that holds it). Where a channel's codes all equal its zero, its
+    // operands are those of that constant row, so the two results are bitwise equal and the
+    // difference is exactly zero. The unit's scale (times 2^24) then multiplies the difference.
+    auto unit_math_sub = [&](const uint4 (&cw)[4], const uint16_t (&sb)[4], const uint4& zw,
+                             const uint4 (&v)[NB][4]) {
+        using O = GsOps<__half>;
+        const uint32_t zl0 = (uint32_t)g * 0x00010001u, zl1 = (uint32_t)(g + 8) * 0x00010001u;
+        const uint32_t zh0 = zl0 << 4, zh1 = zl1 << 4;
+        float clo[NB][4], chi[NB][4], cz[NB][4];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            O::mma_z(clo[b], zl0, zl1, zl0, zl1, v[b][0].x, v[b][0].y);
+            O::mma_z(chi[b], zh0, zh1, zh0, zh1, v[b][0].z, v[b][0].w);
+        }
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                O::mma(clo[b], zl0, zl1, zl0, zl1, v[b][i].x, v[b][i].y);
+                O::mma(chi[b], zh0, zh1, zh0, zh1, v[b][i].z, v[b][i].w);
+            }
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cz[b][e] = fmaf(chi[b][e], 0.0625f, clo[b][e]);
+        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
+            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
+            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+            float alo[NB][4], ahi[NB][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t h0 = mulhi(w0[i], km.m8), h1 = mulhi(w1[i], km.m8);
+                const uint32_t a0 = w0[i] & 0x000F000Fu, a1 = w1[i] & 0x000F000Fu;
+                const uint32_t a2 = h0 & 0x000F000Fu, a3 = h1 & 0x000F000Fu;
+                const uint32_t b0 = w0[i] & 0x00F000F0u, b1 = w1[i] & 0x00F000F0u;
+                const uint32_t b2 = h0 & 0x00F000F0u, b3 = h1 & 0x00F000F0u;
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    if (i == 0) {
+                        O::mma_z(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
+                        O::mma_z(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
+                    } else {
+                        O::mma(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
+                        O::mma(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
+                    }
+                }
+            }
+            const uint32_t z0 = (zws[2 * rt] >> zsh) & 0xFu, z1 = (zws[2 * rt + 1] >> zsh) & 0xFu;
+            const int src0 = (int)(4 * (z0 & 7u)) + t, src1 = (int)(4 * (z1 & 7u)) + t;
+            const float s0 = __half2float(__ushort_as_half(sb[2 * rt])) * 16777216.0f;
+            const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1])) * 16777216.0f;
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                // row g takes row z0 of the constant chains, row g + 8 row z1 (same column 2t, 2t + 1)
+                const float x0 = __shfl_sync(0xffffffffu, cz[b][0], src0);
+                const float x2 = __shfl_sync(0xffffffffu, cz[b][2], src0);
+                const float y0 = __shfl_sync(0xffffffffu, cz[b][0], src1);
+                const float y2 = __shfl_sync(0xffffffffu, cz[b][2], src1);
+                tot[rt][b][0] = fmaf(s0, fmaf(ahi[b][0], 0.0625f, alo[b][0]) - (z0 >= 8u ? x2 : x0), tot[rt][b][0]);
+                tot[rt][b][2] = fmaf(s1, fmaf(ahi[b][2], 0.0625f, alo[b][2]) - (z1 >= 8u ? y2 : y0), tot[rt][b][2]);
+                if (ODD) {
+                    const float x1 = __shfl_sync(0xffffffffu, cz[b][1], src0);
+                    const float x3 = __shfl_sync(0xffffffffu, cz[b][3], src0);
+                    const float y1 = __shfl_sync(0xffffffffu, cz[b][1], src1);
+                    const float y3 = __shfl_sync(0xffffffffu, cz[b][3], src1);
+                    tot[rt][b][1] =
+                        fmaf(s0, fmaf(ahi[b][1], 0.0625f, alo[b][1]) - (z0 >= 8u ? x3 : x1), tot[rt][b][1]);
+                    tot[rt][b][3] =
+                        fmaf(s1, fmaf(ahi[b][3], 0.0625f, alo[b][3]) - (z1 >= 8u ? y3 : y1), tot[rt][b][3]);
+                }
+            }
+        }
+    };
+
     bool aborted = false;
     int s_idx = -1;
     uint32_t ph = 0;
@@ -517,7 +600,9 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         }
         if constexpr (kConv) {
             if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
-            else unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
+            else unit_math_sub(cw, sb, zw, v);
+        } else if constexpr (kPost && std::is_same<T, __half>::value) {
+            unit_math_sub(cw, sb, zw, v);
         } else {
             unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
         }
@@ -525,7 +610,10 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     while (seg_lo < nunits) emit();
 
     // after a timeout: let every copy still in flight land before the CTA exits (a wait that
-    // does not give up on the raised abort flag, still bounded in time)
+    // does not give up on the raised abort flag, still bounded in time). The barrier first: a warp
+    // that completes the count-out of a stage issues its refill, so the copies issued are known
+    // only once every warp has left the loop.
+    __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) {
         volatile int keep_waiting = 0;
         for (int s = 0; s < ns; ++s)

@@ -30,7 +30,7 @@ __global__ void repack_meta_kernel(const uint16_t* __restrict__ scales, const in
                                    int N, int group, TiledLayout L, uint8_t* __restrict__ tiled) {
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t total = (size_t)(K / group) * N;
-    if (idx >= total) return;
+    if (idx >= total) return;   // writes nothing, so nothing to make visible
     const int gi = (int)(idx / N);
     const int n = (int)(idx - (size_t)gi * N);
     const int c = gi / L.groups, gg = gi % L.groups;
@@ -39,6 +39,10 @@ __global__ void repack_meta_kernel(const uint16_t* __restrict__ scales, const in
     *reinterpret_cast<uint16_t*>(rec + L.scales + 256 * gg + 2 * nl) = scales[idx];
     if (zeros && (nl & 7) == 0)
         *reinterpret_cast<int32_t*>(rec + L.zeros + 64 * gg + 4 * (nl / 8)) = zeros[(size_t)gi * (N / 8) + n / 8];
+    // the decode kernel may start on the next launch before this grid has completed (programmatic
+    // dependent launch) and begins streaming weight records before it waits for this grid: every
+    // thread's stores are made visible device-wide before the thread exits
+    __threadfence();
 }
 
 }  // namespace

@@ -44,6 +44,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase with parity `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// try_wait that suspends the thread for at most about `hint_ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -53,20 +79,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Bounded wait for the phase of `bar` with parity `parity` to complete. Gives up after
 // `limit_ns` nanoseconds of waiting or as soon as another thread of the block raised `*abort`;
 // on its own expiry it raises `*abort` and records W4A16_ETIMEOUT in `dev_status`.
-// Returns false when it gave up.
+// Returns false when it gave up. Each try suspends the thread for at most min(limit, 20 us), so
+// the limit is honoured however short it is.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* dev_status, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint32_t hint = limit_ns < 20000ull ? (uint32_t)limit_ns : 20000u;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                *abort = 1;
-                if (dev_status) atomicCAS(dev_status, 0, -7 /* W4A16_ETIMEOUT */);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_for(bar, parity, hint)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            if (dev_status) atomicCAS(dev_status, 0, -7 /* W4A16_ETIMEOUT */);
+            return false;
         }
     }
 }
