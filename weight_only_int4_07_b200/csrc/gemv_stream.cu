@@ -18,22 +18,29 @@
 // lane 0 of each warp leaving a stage counts the warp out on a shared counter, and the warp that
 // completes the count refills the slot with the stage ns positions later, so no warp waits for
 // another to issue a copy. Sixteen warps in four groups: group q takes unit q of every stage,
-// warp w of a group owns channels 32 w .. 32 w + 31 of the unit.
+// warp w of a group owns channels 32 w .. 32 w + 31 of the unit. At the end of a tile one group
+// (rotating over tiles) adds the four groups' sums; the other three hand theirs over through
+// shared memory and an mbarrier and go on without waiting.
 //
 // Math (warp-level tensor-core MMA, m16n8k16, FP32 accumulators), per warp and unit: lane
 // (g = lane / 4, t = lane % 4) reads the 16 bytes of block t (32 K) of channels 32 w + g + 8 r,
 // r = 0..3 (block t keeps channel n at slot n ^ 2t: the four lanes t of a channel hit different
-// banks), and the unit's activations of batch rows 8 b + g. Nibble pairs become 16-bit operands
-// by one mask-OR with a magic exponent: fp16 0x6400 | u = 1024 + u, and for the nibble one
-// position up 0x6400 | (u << 4) = 1024 + 16 u (no shift); bf16 0x4300 | u = 128 + u. The zero
-// point is subtracted exactly in 16 bits: (1024 + u) - (1024 + z), (1024 + 16 u) / 16 - (64 + z),
-// (128 + u) - (128 + z). Group 128: the MMAs accumulate sum a (u - z) of the unit in FP32, and
-// the unit's scale multiplies that sum once. Groups 64 and 32 (a lane's 32 K may span several
-// groups): each operand is scaled first, (u - z) * s rounded once to the 16-bit type (bf16:
-// s = s_hi + s_lo, both exact in bf16), and the MMAs accumulate the whole tile segment.
-// Every mbarrier wait is bounded (2 s); on expiry the kernel records W4A16_ETIMEOUT, stops
-// issuing copies, still passes every CTA barrier and tile counter, and lets the copies in
-// flight land before it exits.
+// banks), and the unit's activations of batch rows 8 b + g.
+//   Group 128 on the fp16 arithmetic (fp16 rows, and bf16 rows converted exactly, below): each
+//   operand register is one AND of a packed word, which leaves the codes as fp16 subnormals
+//   u 2^-24 (or 16 u 2^-24 for the nibble one position up), multiplied exactly by the MMA; the
+//   zero point comes off the FP32 sums with the same MMA chains run on constant rows j 2^-24,
+//   j = 0..15 (each channel takes the row of its zero), and the unit's scale multiplies the
+//   result once.
+//   Otherwise nibble pairs become 16-bit operands by one mask-OR with a magic exponent (fp16
+//   0x6400 | u = 1024 + u, 0x6400 | (u << 4) = 1024 + 16 u; bf16 0x4300 | u = 128 + u) and the
+//   zero point is subtracted exactly in 16 bits: group 128 scales the unit's FP32 sum once;
+//   groups 64 and 32 (a lane's 32 K may span several groups) scale each operand first,
+//   (u - z) * s rounded once to the 16-bit type (bf16: s = s_hi + s_lo, both exact in bf16),
+//   and the MMAs accumulate the whole tile segment.
+// Every wait is bounded (the limit of w4a16_set_wait_limit_ns, 2 s by default); on expiry the
+// kernel records W4A16_ETIMEOUT, stops issuing copies, still passes every barrier and tile
+// counter, and lets the copies in flight land before it exits.
 #include <mutex>
 #include <type_traits>
 
@@ -124,7 +131,9 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     int* rowmin = reinterpret_cast<int*>(zrow + 384);                     // [16] smallest nonzero one
     uint8_t* stages = zrow + kGsZrowBytes;                                // ns x stage_bytes
     uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);
-    int* flags = reinterpret_cast<int*>(full + ns);
+    uint64_t* red_full = full + ns;     // [2] the three other groups' sums of a tile are in `red`
+    uint64_t* red_empty = red_full + 2; // [2] the summing group has read them
+    int* flags = reinterpret_cast<int*>(red_empty + 2);
     volatile int* abort_flag = flags;
     int* issued = flags + 2;            // [ns] copies issued into each slot
     int* leave = flags + 2 + ns;        // [ns] warps that have left the slot's current stage
@@ -134,6 +143,10 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
             mbar_init(&full[i], 1);
             issued[i] = 0;
             leave[i] = 0;
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&red_full[i], 3 * kGsGroupWarps);
+            mbar_init(&red_empty[i], kGsGroupWarps);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -280,12 +293,21 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     int seg_lo = 0, sp_lo = (int)(u0 - (long long)tile * steps);
     int seg_hi = (steps - sp_lo) < nunits ? (steps - sp_lo) : nunits;
 
-    // end of a tile segment: groups 1..3 hand their sums to group 0 through shared memory (two
-    // buffers, by tile parity, so one CTA barrier per tile suffices); group 0 writes C, or this
-    // CTA's partial sums when the tile is cut between CTAs
+    // end of a tile segment: the tile's sums are split over the four groups (each summed the
+    // units it took). One group -- it rotates from tile to tile, so the extra work is shared --
+    // adds them and writes C, or this CTA's partial sums when the tile is cut between CTAs. The
+    // other three write their sums to one of two shared buffers, arrive on its barrier and go on
+    // with the next tile without waiting; they wait (normally long satisfied) only before they
+    // reuse that buffer two tiles later, until its reader has arrived on its `empty` barrier.
+    int n_emit = 0;
     auto emit = [&]() {
-        float* rb = red + (size_t)(tile & 1) * 3 * M * 128;
-        if (grp > 0) {
+        const int bsel = n_emit & 1;
+        const uint32_t use = (uint32_t)(n_emit >> 1) & 1u;   // parity of this buffer's use
+        const int rg = n_emit & 3;                            // the group that sums this tile
+        float* rb = red + (size_t)bsel * 3 * M * 128;
+        if (grp != rg) {
+            const int j = (grp - rg + 3) & 3;                 // 0, 1, 2: its slot in the buffer
+            (void)wait_uniform(&red_empty[bsel], use ^ 1u, abort_flag, p.dev_status, p.wait_ns);
 #pragma unroll
             for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
@@ -293,11 +315,12 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                        if (m < M) rb[((grp - 1) * M + m) * 128 + ch] = tot[rt][b][e];
+                        if (m < M) rb[(j * M + m) * 128 + ch] = tot[rt][b][e];
                     }
-        }
-        __syncthreads();
-        if (grp == 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_full[bsel]);
+        } else {
+            (void)wait_uniform(&red_full[bsel], use, abort_flag, p.dev_status, p.wait_ns);
             T* C = static_cast<T*>(p.C);
             const size_t n0 = (size_t)tile * 128;
             const int cf = unit_owner((long long)tile * steps, U, P);
@@ -314,12 +337,15 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                                                      rb[(2 * M + m) * 128 + ch]
                                                : 0.0f;
                     }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[bsel]);
+            const bool first = wg == 0 && lane == 0;   // the first thread of this group
             if (cf == cl || cta == cf) {
                 if (cf != cl) {
                     // the tile is cut between CTAs cf .. cl and this is cf: the tile is the last of
                     // its range. Wait until every later CTA of the tile has published its sums (they
                     // hold the tile at the start of their ranges), then add them in CTA order.
-                    if (threadIdx.x == 0) {
+                    if (first) {
                         const uint64_t t0 = globaltimer_ns();
                         for (;;) {
                             int n;
@@ -334,7 +360,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                         }
                         p.counters[tile] = 0;
                     }
-                    named_bar(2, 32 * kGsGroupWarps);
+                    named_bar(2 + grp, 32 * kGsGroupWarps);
                     // the loads of up to kPL contributors are in flight together; the sums are
                     // added in CTA order
                     constexpr int kPL = NB == 1 ? 4 : 2;
@@ -394,11 +420,13 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
                             const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
                             if (m < M) part[m * 128 + ch] = vals[rt][b][e];
                         }
-                named_bar(2, 32 * kGsGroupWarps);
-                if (threadIdx.x == 0)
+                __threadfence();
+                named_bar(2 + grp, 32 * kGsGroupWarps);
+                if (first)
                     asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + tile) : "memory");
             }
         }
+        ++n_emit;
         zero_tot();
         ++tile;
         sp_lo = 0;
