@@ -45,9 +45,13 @@ def _layer(K, N, group, sym, seed):
     return (oc, os_, oz), native.w4a16_repack(gc, gs, gz, K, N, group, sym)
 
 
-@pytest.mark.parametrize("how", ["limit", "counters"])
-@pytest.mark.parametrize("M,kernel", [(1, native.KERNEL_GEMV), (8, native.KERNEL_GEMV),
-                                      (64, native.KERNEL_TC), (256, native.KERNEL_TC)])
+# The 1 ns limit runs out for certain only where a wait comes before any copy can have landed:
+# the tensor-core kernel's dequant warps wait for their first weight records at once. The decode
+# kernel first stages A, by which time its first weight stages may already be there, so it is
+# driven to a timeout through its tile counters instead.
+@pytest.mark.parametrize("M,kernel,how", [(1, native.KERNEL_GEMV, "counters"), (8, native.KERNEL_GEMV, "counters"),
+                                          (64, native.KERNEL_TC, "limit"), (64, native.KERNEL_TC, "counters"),
+                                          (256, native.KERNEL_TC, "limit"), (256, native.KERNEL_TC, "counters")])
 def test_waits_run_out_then_the_device_recovers(M, kernel, how):
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     (oc, os_, oz), tiled = _layer(K, N, group, sym, 21)

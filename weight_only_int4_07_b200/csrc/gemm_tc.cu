@@ -25,19 +25,25 @@
 // Warp roles (512 threads):
 //   warp 0      : weight loader -- one bulk copy per two unit records (codes, scales and zeros
 //                 of 2 x 128 K, contiguous in the tiled buffer) into a ring of record slots.
-//   warp 1      : activation loader -- one TMA tile (BN rows x 64 K) per 64-K step into a ring;
-//                 owns the tensor memory allocation.
+//   warp 1      : activation loader -- one TMA tile (BN rows x 64 K) per 64-K step into a deep
+//                 ring (up to 16 slots: the tiles come from L2 and the ring must cover its
+//                 latency plus the MMAs that still read a slot); owns the tensor memory.
 //   warp 2      : MMA issuer -- one thread issues the four tcgen05.mma (K = 16 each) of a 64-K
-//                 step and commits them to the barriers that free the step's two operand slots;
+//                 step, operand A (the weights) from tensor memory and B (the activations) from
+//                 shared memory, and commits them to the barriers that free the step's two slots;
 //                 after a tile's last step it commits the accumulator.
 //   warps 4..7  : epilogue -- tcgen05.ld of the accumulator (warp w reads lanes 32 (w % 4) ..),
-//                 then C (or the published partial sums of a cut tile); two accumulators in
-//                 tensor memory, so one tile's epilogue runs under the next tile's MMAs.
+//                 then C (or the published partial sums of a cut tile); with BN <= 128 two
+//                 accumulators, so one tile's epilogue runs under the next tile's MMAs.
 //   warps 8..15 : dequantize -- thread (n, hh) turns the 32 codes of channel n in block
 //                 2 s + hh of a unit (s = 64-K half) into 16-bit weights (u - z) s (one rounding)
-//                 and writes them into the step's weight tile (128-byte-swizzled, K-major).
+//                 and stores them with tcgen05.st into a ring of weight tiles in tensor memory
+//                 (lane n = channel n, 32 columns of K pairs per 64-K step); warp w writes the
+//                 lanes 32 (w % 4) .. its channels occupy.
+// Tensor memory (512 columns): the accumulators (BN columns each), then the weight-tile ring.
 // Record slots are freed by the dequant warps, activation and weight-tile slots by the MMA
-// commits, so the weight stream runs several units ahead of the tensor cores.
+// commits, so the weight stream runs several units ahead of the tensor cores, and the shared
+// memory holds only copies in flight (weight records and activation tiles).
 // Every wait on an mbarrier or a tile counter is bounded; on expiry the kernel records
 // W4A16_ETIMEOUT in dev_status, every role stops, the loaders wait for their copies in flight,
 // the MMA thread waits for its last MMAs, and the CTA frees its tensor memory and returns.
@@ -61,9 +67,20 @@ constexpr int kTcThreads = 512;
 constexpr int kTcWarpLoadW = 0, kTcWarpLoadA = 1, kTcWarpMma = 2, kTcWarpEpi = 4, kTcWarpDeq = 8;
 constexpr int kTcDeqWarps = 8;
 constexpr int kTcUnitsPerLoad = 2;     // unit records per record slot (one bulk copy)
-constexpr int kTcDTile = 128 * 128;    // weight tile of one 64-K step: 128 channels x 128 B
+constexpr int kTcDCols = 32;           // tensor-memory columns of one 64-K weight tile (K pairs)
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcMaxRing = 16;
+constexpr int kTcTmemCols = 512;
+
+// Accumulators in tensor memory: two (double-buffered) up to BN = 128, one at BN = 256.
+__host__ __device__ constexpr int tc_acc_bufs(int bn) { return bn <= 128 ? 2 : 1; }
+__host__ __device__ constexpr int tc_acc_cols(int bn) { return bn < 32 ? 32 : bn; }
+// weight-tile slots that fit in tensor memory beside the accumulators (at most 8)
+__host__ __device__ constexpr int tc_d_slots(int bn) {
+    return (kTcTmemCols - tc_acc_bufs(bn) * tc_acc_cols(bn)) / kTcDCols > 8
+               ? 8
+               : (kTcTmemCols - tc_acc_bufs(bn) * tc_acc_cols(bn)) / kTcDCols;
+}
 constexpr uint64_t kTcDrainNs = 2000000000ull;
 
 struct TcParams {
@@ -74,8 +91,8 @@ struct TcParams {
     int* dev_status;
     int M, K, N, sym, group;
     uint32_t record, scales_off, zeros_off, slot_w;
-    int P, mblocks, nr, na, nd;
-    uint32_t off_a, off_w, off_bar;   // shared-memory offsets; the weight-tile ring starts at 0
+    int P, mblocks, nr, na;
+    uint32_t off_w, off_bar;   // shared-memory offsets; the activation ring starts at 0
     uint64_t wait_ns;
     GsMasks km;
 };
@@ -96,33 +113,19 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, dev_status, ns));
 }
 
-// Four K-consecutive MMAs D (+)= A . B^T (descriptors advanced by 32 bytes of K each), no commit.
-__device__ __forceinline__ void mma4_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, t;\n\t"
-        "setp.ne.b32 p, %2, 0;\n\t"
-        "setp.eq.b32 t, %1, %1;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %1, p;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %1, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %1, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %1, t;\n\t}" ::"r"(d_tmem),
-        "r"(idesc), "r"(accumulate), "l"(a_desc), "l"(b_desc), "l"(a_desc + 2), "l"(b_desc + 2), "l"(a_desc + 4),
-        "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
-        : "memory");
-}
-
 template <int BN, typename T>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     using Ops = GsOps<T>;
-    constexpr int kCols = BN < 32 ? 32 : BN;     // tensor-memory columns of one accumulator
+    constexpr int kCols = tc_acc_cols(BN);       // tensor-memory columns of one accumulator
+    constexpr int kAcc = tc_acc_bufs(BN);
+    constexpr int kND = tc_d_slots(BN);           // weight-tile slots in tensor memory
     constexpr uint32_t kSlotA = (uint32_t)BN * 128u;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int nr = p.nr, na = p.na, nd = p.nd;
-    uint8_t* ring_d = smem;
-    uint8_t* ring_a = smem + p.off_a;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base, kept a shared-memory pointer (no integer round trip)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int nr = p.nr, na = p.na, nd = kND;
+    uint8_t* ring_a = smem;
     uint8_t* ring_w = smem + p.off_w;
     uint64_t* full_r = reinterpret_cast<uint64_t*>(smem + p.off_bar);
     uint64_t* empty_r = full_r + nr;
@@ -167,7 +170,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         fence_mbar_init();
     }
     if (warp == kTcWarpLoadA) {
-        tmem_alloc(tmem_slot, 2 * kCols);
+        tmem_alloc(tmem_slot, kTcTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -253,7 +256,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                             break;
                         }
                         tc_fence_after();
-                        mma4_f16_ss(d_tmem, smem_desc_sw128(smem_u32(ring_d + (size_t)ds * kTcDTile)),
+                        mma4_f16_ts(d_tmem, tmem + (uint32_t)(kAcc * kCols + ds * kTcDCols),
                                     smem_desc_sw128(smem_u32(ring_a + (size_t)as * kSlotA)), idesc, first ? 0u : 1u);
                         mma_commit(&empty_a[as]);
                         mma_commit(&empty_d[ds]);
@@ -271,7 +274,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 if (!ok) break;
                 mma_commit(&accfull[ab]);
                 ++use[ab];
-                ab ^= 1;
+                ab = (ab + 1) % kAcc;
             }
             // the CTA exits only after its last MMAs completed
             mma_commit(lastmma);
@@ -361,7 +364,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[ab]);
             ++use[ab];
-            ab ^= 1;
+            ab = (ab + 1) % kAcc;
         }
     } else if (warp >= kTcWarpDeq) {
         // ------------------------------------------------------------ dequantize
@@ -369,8 +372,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         const int n = dt & 127, hh = dt >> 7;
         const int sym = p.sym, group = p.group;
         const GsMasks km = p.km;
-        const uint32_t swz = (uint32_t)(n & 7);
-        const uint32_t row_off = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
+        // this warp's lanes of tensor memory (its 32 channels), and the columns of its 32-K block
+        const uint32_t d_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(kAcc * kCols + 16 * hh);
         int rs = 0, ds = 0;
         uint32_t rph = 0, dph = 0;
         bool ok = true;
@@ -405,24 +408,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                         ok = false;
                         break;
                     }
+                    tc_fence_after();   // the MMAs that read this slot completed before the stores
                     const uint32_t za = Ops::zz_a(zv[h]), zb = Ops::zz_b(zv[h]);
                     typename Ops::Scale sc;
                     sc.set(sb[h]);
-                    uint8_t* tile = ring_d + (size_t)ds * kTcDTile;
                     const uint32_t words[4] = {cw[h].x, cw[h].y, cw[h].z, cw[h].w};
+                    uint32_t out[16];   // column c: K pair (2 c, 2 c + 1) of the block
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         uint32_t r[4];
                         Ops::unpack(words[w], km, r);
-                        uint4 out;
-                        out.x = sc.apply(Ops::sub_a(r[0], za));
-                        out.y = sc.apply(Ops::sub_b(r[1], zb));
-                        out.z = sc.apply(Ops::sub_a(r[2], za));
-                        out.w = sc.apply(Ops::sub_b(r[3], zb));
-                        const uint32_t j = (uint32_t)(4 * hh + w);   // 16-byte chunk (8 K) of the 64-K row
-                        *reinterpret_cast<uint4*>(tile + row_off + ((j ^ swz) << 4)) = out;
+                        out[4 * w + 0] = sc.apply(Ops::sub_a(r[0], za));
+                        out[4 * w + 1] = sc.apply(Ops::sub_b(r[1], zb));
+                        out[4 * w + 2] = sc.apply(Ops::sub_a(r[2], za));
+                        out[4 * w + 3] = sc.apply(Ops::sub_b(r[3], zb));
                     }
-                    fence_proxy_async_smem();
+                    tmem_st16(d_lane + (uint32_t)(ds * kTcDCols), out);
+                    tmem_st_wait();
+                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_d[ds]);
                     if (++ds == nd) {
@@ -444,7 +447,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     __syncthreads();
     if (warp == kTcWarpLoadA) {
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * kCols);
+        tmem_dealloc(tmem, kTcTmemCols);
     }
 }
 
@@ -515,17 +518,20 @@ TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
     pl.ctas = (int)(units < n_sm ? units : n_sm);
     pl.slot_w = (uint32_t)((kTcUnitsPerLoad * L.record + 127) & ~127u);
     const uint32_t slot_a = (uint32_t)pl.bn * 128u;
-    pl.nd = 3;
-    pl.na = pl.bn >= 256 ? 3 : 4;
+    pl.nd = tc_d_slots(pl.bn);   // in tensor memory
+    // shared memory: activation tiles first (deep: they come from L2, and a slot stays busy until
+    // its MMAs complete), then at least three record slots, then the barriers
     const size_t bars = 1024;   // barriers, tensor-memory slot, abort flag
-    const size_t fixed = 1024 /* alignment */ + (size_t)pl.nd * kTcDTile + (size_t)pl.na * slot_a + bars;
-    if (fixed >= (size_t)kTcSmemMax) return TcPlan{};
-    size_t nr = ((size_t)kTcSmemMax - fixed) / pl.slot_w;
+    const size_t avail = (size_t)kTcSmemMax - 1024 /* alignment */ - bars;
+    int na = kTcMaxRing;
+    while (na > 2 && (size_t)na * slot_a + 3 * (size_t)pl.slot_w > avail) --na;
+    if ((size_t)na * slot_a + 2 * (size_t)pl.slot_w > avail) return TcPlan{};
+    pl.na = na;
+    size_t nr = (avail - (size_t)na * slot_a) / pl.slot_w;
     if (nr > kTcMaxRing) nr = kTcMaxRing;
-    if (nr < 2) return TcPlan{};
     pl.nr = (int)nr;
-    pl.off_a = (uint32_t)pl.nd * kTcDTile;
-    pl.off_w = pl.off_a + (uint32_t)pl.na * slot_a;
+    pl.off_a = 0;
+    pl.off_w = (uint32_t)na * slot_a;
     pl.off_bar = pl.off_w + (uint32_t)pl.nr * pl.slot_w;
     pl.off_bar = (pl.off_bar + 127u) & ~127u;
     pl.smem = 1024 + pl.off_bar + bars;
@@ -591,8 +597,6 @@ int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, 
     prm.mblocks = pl.mblocks;
     prm.nr = pl.nr;
     prm.na = pl.na;
-    prm.nd = pl.nd;
-    prm.off_a = pl.off_a;
     prm.off_w = pl.off_w;
     prm.off_bar = pl.off_bar;
     prm.wait_ns = wait_limit_ns();

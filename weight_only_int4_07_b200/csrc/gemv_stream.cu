@@ -26,18 +26,14 @@
 // (g = lane / 4, t = lane % 4) reads the 16 bytes of block t (32 K) of channels 32 w + g + 8 r,
 // r = 0..3 (block t keeps channel n at slot n ^ 2t: the four lanes t of a channel hit different
 // banks), and the unit's activations of batch rows 8 b + g.
-//   Group 128 on the fp16 arithmetic (fp16 rows, and bf16 rows converted exactly, below): each
-//   operand register is one AND of a packed word, which leaves the codes as fp16 subnormals
-//   u 2^-24 (or 16 u 2^-24 for the nibble one position up), multiplied exactly by the MMA; the
-//   zero point comes off the FP32 sums with the same MMA chains run on constant rows j 2^-24,
-//   j = 0..15 (each channel takes the row of its zero), and the unit's scale multiplies the
-//   result once.
-//   Otherwise nibble pairs become 16-bit operands by one mask-OR with a magic exponent (fp16
-//   0x6400 | u = 1024 + u, 0x6400 | (u << 4) = 1024 + 16 u; bf16 0x4300 | u = 128 + u) and the
-//   zero point is subtracted exactly in 16 bits: group 128 scales the unit's FP32 sum once;
-//   groups 64 and 32 (a lane's 32 K may span several groups) scale each operand first,
-//   (u - z) * s rounded once to the 16-bit type (bf16: s = s_hi + s_lo, both exact in bf16),
-//   and the MMAs accumulate the whole tile segment.
+//   Nibble pairs become 16-bit operands by one mask-OR with a magic exponent (fp16 0x6400 | u =
+//   1024 + u, 0x6400 | (u << 4) = 1024 + 16 u; bf16 0x4300 | u = 128 + u) and the zero point is
+//   subtracted exactly in 16 bits: group 128 scales the unit's FP32 sum once; groups 64 and 32
+//   (a lane's 32 K may span several groups) scale each operand first, (u - z) * s rounded once to
+//   the 16-bit type (bf16: s = s_hi + s_lo, both exact in bf16), and the MMAs accumulate the
+//   whole tile segment. (Codes fed to the MMA as fp16 subnormals u 2^-24, one AND per operand
+//   and the zero point taken off the FP32 sums with extra MMA chains on constant rows, cut the
+//   integer work but added half again as many MMAs, and measured 2% slower.)
 // Every wait is bounded (the limit of w4a16_set_wait_limit_ns, 2 s by default); on expiry the
 // kernel records W4A16_ETIMEOUT, stops issuing copies, still passes every barrier and tile
 // counter, and lets the copies in flight land before it exits.
@@ -54,11 +50,16 @@ namespace {
 
 using namespace sm100;
 
+// Four groups of 4 warps per CTA (each group takes one unit of a stage), one CTA per SM. (Two
+// groups and two CTAs per SM, which let the next launch's CTAs start on an SM before the previous
+// launch has left it, measured 12% slower on the Llama-3-70B-shaped stack.)
 constexpr int kGsGroups = 4, kGsGroupWarps = 4, kGsWarps = kGsGroups * kGsGroupWarps;
+constexpr int kGsCtasPerSm = 1;
 constexpr int kGsThreads = 32 * kGsWarps;
 constexpr int kGsUnitsPerStage = kGsGroups;
+static_assert(kGsGroups >= 2 && kGsGroups <= 4, "two to four groups");
 constexpr int kGsMinStages = 3, kGsMaxStages = 16;
-constexpr int kGsSmemMax = 227 * 1024;
+constexpr int kGsSmemMax = (228 * 1024) / kGsCtasPerSm - 1024;   // per CTA; 1 KiB reserved each
 constexpr uint64_t kGsSpin = 2000000000ull;
 constexpr int kGsZrowBytes = 512;   // the zero activation block, then per-row exponent bounds
 
@@ -101,7 +102,7 @@ struct GsParams {
 
 // NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
 template <int NB, typename T, int GROUP, bool ODD>
-__global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsParams p) {
+__global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(const GsParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     constexpr bool kPost = (GROUP == 128);   // one group per unit: scale the unit's sum
     // bf16 activations at group 128 run the fp16 arithmetic (fewer instructions per weight)
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     const uint32_t R = p.record, stage_bytes = p.stage_bytes, RS = p.row_bytes;
 
     uint8_t* acts = smem_raw;                                             // [M][RS]
-    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][3][M][128]
+    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][groups - 1][M][128]
     uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes;                 // 320 zero bytes
     int* rowexp = reinterpret_cast<int*>(zrow + 320);                     // [16] largest exponent per row
     int* rowmin = reinterpret_cast<int*>(zrow + 384);                     // [16] smallest nonzero one
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
             leave[i] = 0;
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&red_full[i], 3 * kGsGroupWarps);
+            mbar_init(&red_full[i], (kGsGroups - 1) * kGsGroupWarps);
             mbar_init(&red_empty[i], kGsGroupWarps);
         }
         *abort_flag = 0;
@@ -303,10 +304,10 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
     auto emit = [&]() {
         const int bsel = n_emit & 1;
         const uint32_t use = (uint32_t)(n_emit >> 1) & 1u;   // parity of this buffer's use
-        const int rg = n_emit & 3;                            // the group that sums this tile
-        float* rb = red + (size_t)bsel * 3 * M * 128;
+        const int rg = n_emit % kGsGroups;                    // the group that sums this tile
+        float* rb = red + (size_t)bsel * (kGsGroups - 1) * M * 128;
         if (grp != rg) {
-            const int j = (grp - rg + 3) & 3;                 // 0, 1, 2: its slot in the buffer
+            const int j = (grp - rg - 1 + kGsGroups) % kGsGroups;   // its slot in the buffer
             (void)wait_uniform(&red_empty[bsel], use ^ 1u, abort_flag, p.dev_status, p.wait_ns);
 #pragma unroll
             for (int rt = 0; rt < 2; ++rt)
@@ -333,9 +334,10 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                        vals[rt][b][e] = m < M ? tot[rt][b][e] + rb[m * 128 + ch] + rb[(M + m) * 128 + ch] +
-                                                     rb[(2 * M + m) * 128 + ch]
-                                               : 0.0f;
+                        float v = tot[rt][b][e];
+#pragma unroll
+                        for (int j = 0; j < kGsGroups - 1; ++j) v += m < M ? rb[(j * M + m) * 128 + ch] : 0.0f;
+                        vals[rt][b][e] = m < M ? v : 0.0f;
                     }
             __syncwarp();
             if (lane == 0) mbar_arrive(&red_empty[bsel]);
@@ -497,89 +499,6 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         }
     };
 
-    // Group 128 on the fp16 arithmetic: the codes enter the MMAs as fp16 subnormals, u 2^-24 for
-    // the pairs (0, 1) and (4, 5) of a word and 16 u 2^-24 for (2, 3) and (6, 7), each operand
-    // register one AND of the word (no magic, no zero-point arithmetic), summed in two chains
-    // (lo, hi) per row tile. The zero point comes off after the MMAs: per unit the same two chains
-    // run on constant operands whose row j holds j 2^-24 (16 j 2^-24), which gives
-    // sum_k a_k j 2^-24 for every zero j = 0..15, and each channel takes the row of its own zero
-    // (a shuffle from the lane that holds it). Where a channel's codes all equal its zero, its
-    // operands are those of that constant row, so the two results are bitwise equal and the
-    // difference is exactly zero. The unit's scale (times 2^24) then multiplies the difference.
-    auto unit_math_sub = [&](const uint4 (&cw)[4], const uint16_t (&sb)[4], const uint4& zw,
-                             const uint4 (&v)[NB][4]) {
-        using O = GsOps<__half>;
-        const uint32_t zl0 = (uint32_t)g * 0x00010001u, zl1 = (uint32_t)(g + 8) * 0x00010001u;
-        const uint32_t zh0 = zl0 << 4, zh1 = zl1 << 4;
-        float clo[NB][4], chi[NB][4], cz[NB][4];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            O::mma_z(clo[b], zl0, zl1, zl0, zl1, v[b][0].x, v[b][0].y);
-            O::mma_z(chi[b], zh0, zh1, zh0, zh1, v[b][0].z, v[b][0].w);
-        }
-#pragma unroll
-        for (int i = 1; i < 4; ++i)
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                O::mma(clo[b], zl0, zl1, zl0, zl1, v[b][i].x, v[b][i].y);
-                O::mma(chi[b], zh0, zh1, zh0, zh1, v[b][i].z, v[b][i].w);
-            }
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) cz[b][e] = fmaf(chi[b][e], 0.0625f, clo[b][e]);
-        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
-#pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
-            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
-            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
-            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
-            float alo[NB][4], ahi[NB][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t h0 = mulhi(w0[i], km.m8), h1 = mulhi(w1[i], km.m8);
-                const uint32_t a0 = w0[i] & 0x000F000Fu, a1 = w1[i] & 0x000F000Fu;
-                const uint32_t a2 = h0 & 0x000F000Fu, a3 = h1 & 0x000F000Fu;
-                const uint32_t b0 = w0[i] & 0x00F000F0u, b1 = w1[i] & 0x00F000F0u;
-                const uint32_t b2 = h0 & 0x00F000F0u, b3 = h1 & 0x00F000F0u;
-#pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    if (i == 0) {
-                        O::mma_z(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
-                        O::mma_z(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
-                    } else {
-                        O::mma(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
-                        O::mma(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
-                    }
-                }
-            }
-            const uint32_t z0 = (zws[2 * rt] >> zsh) & 0xFu, z1 = (zws[2 * rt + 1] >> zsh) & 0xFu;
-            const int src0 = (int)(4 * (z0 & 7u)) + t, src1 = (int)(4 * (z1 & 7u)) + t;
-            const float s0 = __half2float(__ushort_as_half(sb[2 * rt])) * 16777216.0f;
-            const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1])) * 16777216.0f;
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                // row g takes row z0 of the constant chains, row g + 8 row z1 (same column 2t, 2t + 1)
-                const float x0 = __shfl_sync(0xffffffffu, cz[b][0], src0);
-                const float x2 = __shfl_sync(0xffffffffu, cz[b][2], src0);
-                const float y0 = __shfl_sync(0xffffffffu, cz[b][0], src1);
-                const float y2 = __shfl_sync(0xffffffffu, cz[b][2], src1);
-                tot[rt][b][0] = fmaf(s0, fmaf(ahi[b][0], 0.0625f, alo[b][0]) - (z0 >= 8u ? x2 : x0), tot[rt][b][0]);
-                tot[rt][b][2] = fmaf(s1, fmaf(ahi[b][2], 0.0625f, alo[b][2]) - (z1 >= 8u ? y2 : y0), tot[rt][b][2]);
-                if (ODD) {
-                    const float x1 = __shfl_sync(0xffffffffu, cz[b][1], src0);
-                    const float x3 = __shfl_sync(0xffffffffu, cz[b][3], src0);
-                    const float y1 = __shfl_sync(0xffffffffu, cz[b][1], src1);
-                    const float y3 = __shfl_sync(0xffffffffu, cz[b][3], src1);
-                    tot[rt][b][1] =
-                        fmaf(s0, fmaf(ahi[b][1], 0.0625f, alo[b][1]) - (z0 >= 8u ? x3 : x1), tot[rt][b][1]);
-                    tot[rt][b][3] =
-                        fmaf(s1, fmaf(ahi[b][3], 0.0625f, alo[b][3]) - (z1 >= 8u ? y3 : y1), tot[rt][b][3]);
-                }
-            }
-        }
-    };
-
     bool aborted = false;
     int s_idx = -1;
     uint32_t ph = 0;
@@ -628,9 +547,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_kernel(const GsPara
         }
         if constexpr (kConv) {
             if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
-            else unit_math_sub(cw, sb, zw, v);
-        } else if constexpr (kPost && std::is_same<T, __half>::value) {
-            unit_math_sub(cw, sb, zw, v);
+            else unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
         } else {
             unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
         }
@@ -723,7 +640,7 @@ GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
     const size_t units = (size_t)(Ks / 128);
     pl.row_bytes = 320 * units + ((units & 1) ? 0 : 64);          // 80-byte blocks; rows 64 mod 128 apart
     pl.act_bytes = ((size_t)M * pl.row_bytes + 127) & ~(size_t)127;
-    pl.red_bytes = (size_t)2 * 3 * M * 128 * 4;
+    pl.red_bytes = (size_t)2 * (kGsGroups - 1) * M * 128 * 4;
     pl.stage_bytes = ((size_t)kGsUnitsPerStage * L.record + 127) & ~(size_t)127;
     const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 8 + 8 * kGsMaxStages + 127) & ~(size_t)127;
     const size_t fixed = pl.act_bytes + pl.red_bytes + kGsZrowBytes + flags;
@@ -734,7 +651,8 @@ GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
     pl.ns = (int)ns;
     pl.smem = fixed + ns * pl.stage_bytes;
     const long long total_units = (long long)(N / 128) * (Ks / 128);
-    pl.ctas = n_sm > 0 ? (int)(total_units < n_sm ? total_units : n_sm) : 0;
+    const long long slots = (long long)kGsCtasPerSm * n_sm;
+    pl.ctas = n_sm > 0 ? (int)(total_units < slots ? total_units : slots) : 0;
     pl.ok = pl.ctas > 0;
     return pl;
 }
@@ -753,7 +671,7 @@ GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_s
         pl = plan_slice(M, N, K / S, group, sym, n_sm);
         if (pl.ok) {
             pl.slices = S;
-            pl.partial_bytes = (size_t)2 * (n_sm > 0 ? n_sm : 0) * M * 128 * 4 +
+            pl.partial_bytes = (size_t)2 * kGsCtasPerSm * (n_sm > 0 ? n_sm : 0) * M * 128 * 4 +
                                (S > 1 ? (size_t)S * M * N * 4 : 0);
             return pl;
         }
@@ -776,7 +694,7 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.C = C;
     prm.counters = static_cast<int*>(workspace);
     prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kGemvStreamCounterBytes);
-    float* slice_out = prm.partials + (size_t)2 * sm_count() * M * 128;
+    float* slice_out = prm.partials + (size_t)2 * kGsCtasPerSm * sm_count() * M * 128;
     prm.dev_status = dev_status;
     prm.M = M;
     prm.K = Ks;

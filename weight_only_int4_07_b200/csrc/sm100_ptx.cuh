@@ -268,6 +268,35 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective, 32x32b shape).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// Four K-consecutive MMAs D (+)= A . B^T with A (M = 128 rows in the 128 lanes, 16-bit K pairs
+// per 32-bit column, eight columns per K = 16) read from tensor memory and B from shared memory
+// (descriptor advanced by 32 bytes of K each), no commit. The first MMA accumulates when
+// `accumulate` is non-zero; the other three always accumulate.
+__device__ __forceinline__ void mma4_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %3, 0;\n\t"
+        "setp.eq.b32 t, %2, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %4, %2, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %2, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %2, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %2, t;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(idesc), "r"(accumulate), "l"(b_desc), "r"(a_tmem + 8), "l"(b_desc + 2), "r"(a_tmem + 16),
+        "l"(b_desc + 4), "r"(a_tmem + 24), "l"(b_desc + 6)
+        : "memory");
+}
+
 // ------------------------------------------------------------------------------ clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
