@@ -67,19 +67,16 @@ constexpr int kTcThreads = 512;
 constexpr int kTcWarpLoadW = 0, kTcWarpLoadA = 1, kTcWarpMma = 2, kTcWarpEpi = 4, kTcWarpDeq = 8;
 constexpr int kTcDeqWarps = 8;
 constexpr int kTcUnitsPerLoad = 2;     // unit records per record slot (one bulk copy)
-constexpr int kTcDCols = 32;           // tensor-memory columns of one 64-K weight tile (K pairs)
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcMaxRing = 16;
 constexpr int kTcTmemCols = 512;
+constexpr int kTcStepCols = 64;        // tensor-memory columns of one 128-K weight tile (K pairs)
 
-// Accumulators in tensor memory: two (double-buffered) up to BN = 128, one at BN = 256.
-__host__ __device__ constexpr int tc_acc_bufs(int bn) { return bn <= 128 ? 2 : 1; }
+// Two accumulators (BN columns each, at least 32) in tensor memory, then the step ring's weight
+// tiles: as many as fit, at most 8.
 __host__ __device__ constexpr int tc_acc_cols(int bn) { return bn < 32 ? 32 : bn; }
-// weight-tile slots that fit in tensor memory beside the accumulators (at most 8)
-__host__ __device__ constexpr int tc_d_slots(int bn) {
-    return (kTcTmemCols - tc_acc_bufs(bn) * tc_acc_cols(bn)) / kTcDCols > 8
-               ? 8
-               : (kTcTmemCols - tc_acc_bufs(bn) * tc_acc_cols(bn)) / kTcDCols;
+__host__ __device__ constexpr int tc_steps(int bn) {
+    return (kTcTmemCols - 2 * tc_acc_cols(bn)) / kTcStepCols > 8 ? 8 : (kTcTmemCols - 2 * tc_acc_cols(bn)) / kTcStepCols;
 }
 constexpr uint64_t kTcDrainNs = 2000000000ull;
 
@@ -91,8 +88,8 @@ struct TcParams {
     int* dev_status;
     int M, K, N, sym, group;
     uint32_t record, scales_off, zeros_off, slot_w;
-    int P, mblocks, nr, na;
-    uint32_t off_w, off_bar;   // shared-memory offsets; the activation ring starts at 0
+    int P, mblocks, nr;
+    uint32_t off_w, off_bar;   // shared-memory offsets; the activation tiles start at 0
     uint64_t wait_ns;
     GsMasks km;
 };
@@ -118,22 +115,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     using Ops = GsOps<T>;
     constexpr int kCols = tc_acc_cols(BN);       // tensor-memory columns of one accumulator
-    constexpr int kAcc = tc_acc_bufs(BN);
-    constexpr int kND = tc_d_slots(BN);           // weight-tile slots in tensor memory
-    constexpr uint32_t kSlotA = (uint32_t)BN * 128u;
+    constexpr int NS = tc_steps(BN);             // steps in flight (activation + weight tiles)
+    constexpr uint32_t kSlotA = (uint32_t)BN * 256u;   // 128 K of BN rows: two 64-K TMA boxes
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, kept a shared-memory pointer (no integer round trip)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int nr = p.nr, na = p.na, nd = kND;
+    const int nr = p.nr;
     uint8_t* ring_a = smem;
     uint8_t* ring_w = smem + p.off_w;
     uint64_t* full_r = reinterpret_cast<uint64_t*>(smem + p.off_bar);
     uint64_t* empty_r = full_r + nr;
-    uint64_t* full_a = empty_r + nr;
-    uint64_t* empty_a = full_a + na;
-    uint64_t* full_d = empty_a + na;
-    uint64_t* empty_d = full_d + nd;
-    uint64_t* accfull = empty_d + nd;    // [2]
+    uint64_t* full_a = empty_r + nr;     // [NS] the step's activation tile landed
+    uint64_t* full_d = full_a + NS;      // [NS] the step's weight tile is in tensor memory
+    uint64_t* free_s = full_d + NS;      // [NS] the step's MMAs completed: both tiles free
+    uint64_t* accfull = free_s + NS;     // [2]
     uint64_t* accempty = accfull + 2;    // [2]
     uint64_t* lastmma = accempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lastmma + 1);
@@ -153,13 +148,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             mbar_init(&full_r[i], 1);
             mbar_init(&empty_r[i], kTcDeqWarps);
         }
-        for (int i = 0; i < na; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&full_a[i], 1);
-            mbar_init(&empty_a[i], 1);
-        }
-        for (int i = 0; i < nd; ++i) {
             mbar_init(&full_d[i], kTcDeqWarps);
-            mbar_init(&empty_d[i], 1);
+            mbar_init(&free_s[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accfull[i], 1);
@@ -177,6 +169,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_w = tmem + (uint32_t)(2 * kCols);   // the step ring's weight tiles
 
     if (warp == kTcWarpLoadW) {
         // ------------------------------------------------------------ weight records
@@ -208,38 +201,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         // ------------------------------------------------------------ activation tiles
         if (lane == 0) {
             prefetch_tensormap(&tmA);
-            int as = 0, issued[kTcMaxRing];
-            uint32_t aph = 0;
-            bool ok = true;
-            for (int i = 0; i < na; ++i) issued[i] = 0;
-            for (long long i = u0; i < u1 && ok; ++i) {
+            int issued[8];
+            for (int i = 0; i < NS; ++i) issued[i] = 0;
+            int s = 0;
+            uint32_t ph = 0;
+            for (long long i = u0; i < u1; ++i) {
                 const long long tau = i / UT;
                 const int mb = (int)(tau % p.mblocks);
                 const int ku = (int)(i - tau * UT);
-                for (int h = 0; h < 2; ++h) {
-                    if (!mbar_wait(&empty_a[as], aph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full_a[as], kSlotA);
-                    tma_2d_g2s(ring_a + (size_t)as * kSlotA, &tmA, ku * 128 + h * 64, mb * BN, &full_a[as]);
-                    ++issued[as];
-                    if (++as == na) {
-                        as = 0;
-                        aph ^= 1u;
-                    }
+                if (!mbar_wait(&free_s[s], ph ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
+                mbar_arrive_expect_tx(&full_a[s], kSlotA);
+                uint8_t* dst = ring_a + (size_t)s * kSlotA;
+                tma_2d_g2s(dst, &tmA, ku * 128, mb * BN, &full_a[s]);
+                tma_2d_g2s(dst + kSlotA / 2, &tmA, ku * 128 + 64, mb * BN, &full_a[s]);
+                ++issued[s];
+                if (++s == NS) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
             volatile int keep = 0;
-            for (int s = 0; s < na; ++s)
-                if (issued[s] > 0) mbar_wait(&full_a[s], (uint32_t)(issued[s] - 1) & 1u, &keep, nullptr, kTcDrainNs);
+            for (int q = 0; q < NS; ++q)
+                if (issued[q] > 0) mbar_wait(&full_a[q], (uint32_t)(issued[q] - 1) & 1u, &keep, nullptr, kTcDrainNs);
         }
     } else if (warp == kTcWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_f16(BN, std::is_same<T, __nv_bfloat16>::value);
-            int as = 0, ds = 0, use[2] = {0, 0}, ab = 0;
-            uint32_t aph = 0, dph = 0;
+            int s = 0, use[2] = {0, 0}, ab = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (long long i = u0; i < u1 && ok;) {
                 const long long tau = i / UT;
@@ -248,33 +238,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(ab * kCols);
                 bool first = true;
-                for (; i < seg_end && ok; ++i) {
-                    for (int h = 0; h < 2; ++h) {
-                        if (!mbar_wait(&full_d[ds], dph, abort_flag, p.dev_status, wait_ns) ||
-                            !mbar_wait(&full_a[as], aph, abort_flag, p.dev_status, wait_ns)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        mma4_f16_ts(d_tmem, tmem + (uint32_t)(kAcc * kCols + ds * kTcDCols),
-                                    smem_desc_sw128(smem_u32(ring_a + (size_t)as * kSlotA)), idesc, first ? 0u : 1u);
-                        mma_commit(&empty_a[as]);
-                        mma_commit(&empty_d[ds]);
-                        first = false;
-                        if (++as == na) {
-                            as = 0;
-                            aph ^= 1u;
-                        }
-                        if (++ds == nd) {
-                            ds = 0;
-                            dph ^= 1u;
-                        }
+                for (; i < seg_end; ++i) {
+                    if (!mbar_wait(&full_d[s], ph, abort_flag, p.dev_status, wait_ns) ||
+                        !mbar_wait(&full_a[s], ph, abort_flag, p.dev_status, wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // the unit's eight K-steps of 16: weights from tensor memory, activations from
+                    // the two 64-K boxes of the step's tile; one commit frees both tiles
+                    const uint32_t a_tm = tmem_w + (uint32_t)(s * kTcStepCols);
+                    const uint32_t b_sm = smem_u32(ring_a + (size_t)s * kSlotA);
+                    mma4_f16_ts(d_tmem, a_tm, smem_desc_sw128(b_sm), idesc, first ? 0u : 1u);
+                    mma4_f16_ts(d_tmem, a_tm + 32u, smem_desc_sw128(b_sm + kSlotA / 2), idesc, 1u);
+                    mma_commit(&free_s[s]);
+                    first = false;
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
                     }
                 }
                 if (!ok) break;
                 mma_commit(&accfull[ab]);
                 ++use[ab];
-                ab = (ab + 1) % kAcc;
+                ab ^= 1;
             }
             // the CTA exits only after its last MMAs completed
             mma_commit(lastmma);
@@ -327,15 +314,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                         uint32_t v[16];
                         tmem_ld16(lane_base + (uint32_t)(c * 16), v);
                         tmem_ld_wait();
+                        float y[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(v[j]);
+                        // the other CTAs' sums, in CTA order; the 16 loads of one CTA in flight together
+#pragma unroll 1
+                        for (int cc = cf + 1; cc <= cl; ++cc) {
+                            const float* part = p.partials + ((size_t)cc * BN + c * 16) * 128 + n;
+                            float pv[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pv[j] = m0 + c * 16 + j < p.M ? __ldcg(part + j * 128) : 0.0f;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) y[j] += pv[j];
+                        }
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const int mr = c * 16 + j, m = m0 + mr;
-                            if (m < p.M) {
-                                float y = __uint_as_float(v[j]);
-                                for (int cc = cf + 1; cc <= cl; ++cc)
-                                    y += __ldcg(p.partials + ((size_t)cc * BN + mr) * 128 + n);
-                                C[(size_t)m * p.N + n0 + n] = Act<T>::from_f32(y);
-                            }
+                            const int m = m0 + c * 16 + j;
+                            if (m < p.M) C[(size_t)m * p.N + n0 + n] = Act<T>::from_f32(y[j]);
                         }
                     }
                 }
@@ -364,7 +359,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[ab]);
             ++use[ab];
-            ab = (ab + 1) % kAcc;
+            ab ^= 1;
         }
     } else if (warp >= kTcWarpDeq) {
         // ------------------------------------------------------------ dequantize
@@ -372,10 +367,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         const int n = dt & 127, hh = dt >> 7;
         const int sym = p.sym, group = p.group;
         const GsMasks km = p.km;
-        // this warp's lanes of tensor memory (its 32 channels), and the columns of its 32-K block
-        const uint32_t d_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(kAcc * kCols + 16 * hh);
-        int rs = 0, ds = 0;
-        uint32_t rph = 0, dph = 0;
+        // this warp's lanes of tensor memory (its 32 channels); the thread writes 32-K blocks hh and
+        // 2 + hh of each unit, columns [16 hh, 16 hh + 16) and [32 + 16 hh, + 16) of the step's tile
+        const uint32_t d_lane = tmem_w + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(16 * hh);
+        int rs = 0, s = 0;
+        uint32_t rph = 0, ph = 0;
         bool ok = true;
         for (long long i = u0; i < u1 && ok;) {
             const long long tau = i / UT;
@@ -386,9 +382,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 ok = false;
                 break;
             }
-            for (int uu = 0; uu < nu && ok; ++uu) {
+            for (int uu = 0; uu < nu; ++uu) {
                 const uint8_t* rec = ring_w + (size_t)rs * p.slot_w + (size_t)uu * R;
-                // this thread's 32-K blocks of the unit's two 64-K halves, with their scale and zero
                 uint4 cw[2];
                 uint16_t sb[2];
                 uint32_t zv[2];
@@ -402,13 +397,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                                 : (*reinterpret_cast<const uint32_t*>(rec + p.zeros_off + 64 * lg + 4 * (n >> 3)) >>
                                    (4 * (n & 7))) & 0xFu;
                 }
+                if (!tc_wait(&free_s[s], ph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();   // the MMAs that read this tile completed before the stores
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if (!tc_wait(&empty_d[ds], dph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();   // the MMAs that read this slot completed before the stores
                     const uint32_t za = Ops::zz_a(zv[h]), zb = Ops::zz_b(zv[h]);
                     typename Ops::Scale sc;
                     sc.set(sb[h]);
@@ -423,15 +418,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                         out[4 * w + 2] = sc.apply(Ops::sub_a(r[2], za));
                         out[4 * w + 3] = sc.apply(Ops::sub_b(r[3], zb));
                     }
-                    tmem_st16(d_lane + (uint32_t)(ds * kTcDCols), out);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full_d[ds]);
-                    if (++ds == nd) {
-                        ds = 0;
-                        dph ^= 1u;
-                    }
+                    tmem_st16(d_lane + (uint32_t)(s * kTcStepCols + 32 * h), out);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_d[s]);
+                if (++s == NS) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
             __syncwarp();
@@ -502,8 +497,7 @@ int tc_block_rows(int M) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return 64;
-    if (M <= 128) return 128;
-    return 256;
+    return 128;   // more rows: several blocks of 128 (two accumulators of 128 columns in TMEM)
 }
 
 TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
@@ -517,21 +511,17 @@ TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
     const long long units = tiles * (K / 128);
     pl.ctas = (int)(units < n_sm ? units : n_sm);
     pl.slot_w = (uint32_t)((kTcUnitsPerLoad * L.record + 127) & ~127u);
-    const uint32_t slot_a = (uint32_t)pl.bn * 128u;
-    pl.nd = tc_d_slots(pl.bn);   // in tensor memory
-    // shared memory: activation tiles first (deep: they come from L2, and a slot stays busy until
-    // its MMAs complete), then at least three record slots, then the barriers
+    pl.nd = tc_steps(pl.bn);   // steps in flight: activation tiles in shared memory, weights in TMEM
+    pl.na = pl.nd;
+    const uint32_t slot_a = (uint32_t)pl.bn * 256u;
     const size_t bars = 1024;   // barriers, tensor-memory slot, abort flag
     const size_t avail = (size_t)kTcSmemMax - 1024 /* alignment */ - bars;
-    int na = kTcMaxRing;
-    while (na > 2 && (size_t)na * slot_a + 3 * (size_t)pl.slot_w > avail) --na;
-    if ((size_t)na * slot_a + 2 * (size_t)pl.slot_w > avail) return TcPlan{};
-    pl.na = na;
-    size_t nr = (avail - (size_t)na * slot_a) / pl.slot_w;
+    if ((size_t)pl.na * slot_a + 2 * (size_t)pl.slot_w > avail) return TcPlan{};
+    size_t nr = (avail - (size_t)pl.na * slot_a) / pl.slot_w;
     if (nr > kTcMaxRing) nr = kTcMaxRing;
     pl.nr = (int)nr;
     pl.off_a = 0;
-    pl.off_w = (uint32_t)na * slot_a;
+    pl.off_w = (uint32_t)pl.na * slot_a;
     pl.off_bar = pl.off_w + (uint32_t)pl.nr * pl.slot_w;
     pl.off_bar = (pl.off_bar + 127u) & ~127u;
     pl.smem = 1024 + pl.off_bar + bars;
@@ -562,7 +552,6 @@ int launch_tc_bn(int bn, const CUtensorMap& map, const TcParams& prm, size_t sme
         case 32: return launch_tc_typed<32, T>(map, prm, smem, stream);
         case 64: return launch_tc_typed<64, T>(map, prm, smem, stream);
         case 128: return launch_tc_typed<128, T>(map, prm, smem, stream);
-        case 256: return launch_tc_typed<256, T>(map, prm, smem, stream);
         default: return W4A16_EUNSUPPORTED;
     }
 }
@@ -596,7 +585,6 @@ int launch_gemm_tc(const void* A, int a_dtype, int M, int K, const void* tiled, 
     prm.P = pl.ctas;
     prm.mblocks = pl.mblocks;
     prm.nr = pl.nr;
-    prm.na = pl.na;
     prm.off_w = pl.off_w;
     prm.off_bar = pl.off_bar;
     prm.wait_ns = wait_limit_ns();
