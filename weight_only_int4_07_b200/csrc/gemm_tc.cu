@@ -22,25 +22,27 @@
 // waits for the count (acquire, bounded), adds the sums in CTA order, writes C and resets the
 // counter. The result does not depend on timing.
 //
-// Warp roles (512 threads):
+// Warp roles (768 threads):
 //   warp 0      : weight loader -- one bulk copy per two unit records (codes, scales and zeros
 //                 of 2 x 128 K, contiguous in the tiled buffer) into a ring of record slots.
-//   warp 1      : activation loader -- one TMA tile (BN rows x 64 K) per 64-K step into a deep
-//                 ring (up to 16 slots: the tiles come from L2 and the ring must cover its
-//                 latency plus the MMAs that still read a slot); owns the tensor memory.
-//   warp 2      : MMA issuer -- one thread issues the four tcgen05.mma (K = 16 each) of a 64-K
-//                 step, operand A (the weights) from tensor memory and B (the activations) from
-//                 shared memory, and commits them to the barriers that free the step's two slots;
-//                 after a tile's last step it commits the accumulator.
+//   warp 1      : activation loader -- per 128-K step (one unit), two TMA boxes of BN rows x
+//                 64 K into the step's slot of a ring (4-7 slots: the tiles come from L2, and a
+//                 slot stays busy until its MMAs complete); owns the tensor memory.
+//   warp 2      : MMA issuer -- one thread issues the eight tcgen05.mma (K = 16 each) of a step,
+//                 operand A (the weights) from tensor memory and B (the activations) from shared
+//                 memory, and one commit that frees the step's activation and weight tiles
+//                 together; after a tile's last step a commit to the accumulator.
 //   warps 4..7  : epilogue -- tcgen05.ld of the accumulator (warp w reads lanes 32 (w % 4) ..),
-//                 then C (or the published partial sums of a cut tile); with BN <= 128 two
-//                 accumulators, so one tile's epilogue runs under the next tile's MMAs.
-//   warps 8..15 : dequantize -- thread (n, hh) turns the 32 codes of channel n in block
-//                 2 s + hh of a unit (s = 64-K half) into 16-bit weights (u - z) s (one rounding)
-//                 and stores them with tcgen05.st into a ring of weight tiles in tensor memory
-//                 (lane n = channel n, 32 columns of K pairs per 64-K step); warp w writes the
-//                 lanes 32 (w % 4) .. its channels occupy.
-// Tensor memory (512 columns): the accumulators (BN columns each), then the weight-tile ring.
+//                 then C (or the published partial sums of a cut tile); two accumulators, so one
+//                 tile's epilogue runs under the next tile's MMAs.
+//   warps 8..23 : dequantize -- thread (n, b) turns the 32 codes of channel n in 32-K block b
+//                 of a unit into 16-bit weights (u - z) s (one rounding) and stores them with
+//                 tcgen05.st into a ring of weight tiles in tensor memory (lane n = channel n, 64
+//                 columns of K pairs per 128-K step); warp w writes the lanes 32 (w % 4) .. its
+//                 channels occupy.
+// Tensor memory (512 columns): two accumulators (BN <= 128 columns each), then the weight tiles
+// of the step ring (64 columns per step). A has at most 128 rows per tile; more rows of A are
+// more tiles (row blocks), whose weights are dequantized again but read from L2.
 // Record slots are freed by the dequant warps, activation and weight-tile slots by the MMA
 // commits, so the weight stream runs several units ahead of the tensor cores, and the shared
 // memory holds only copies in flight (weight records and activation tiles).
@@ -63,9 +65,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 512;
+constexpr int kTcThreads = 768;
 constexpr int kTcWarpLoadW = 0, kTcWarpLoadA = 1, kTcWarpMma = 2, kTcWarpEpi = 4, kTcWarpDeq = 8;
-constexpr int kTcDeqWarps = 8;
+constexpr int kTcDeqWarps = 16;
 constexpr int kTcUnitsPerLoad = 2;     // unit records per record slot (one bulk copy)
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcMaxRing = 16;
@@ -364,12 +366,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     } else if (warp >= kTcWarpDeq) {
         // ------------------------------------------------------------ dequantize
         const int dt = threadIdx.x - 32 * kTcWarpDeq;
-        const int n = dt & 127, hh = dt >> 7;
-        const int sym = p.sym, group = p.group;
+        const int n = dt & 127, blk = dt >> 7;   // channel, and the unit's 32-K block (0..3)
+        const int sym = p.sym;
         const GsMasks km = p.km;
-        // this warp's lanes of tensor memory (its 32 channels); the thread writes 32-K blocks hh and
-        // 2 + hh of each unit, columns [16 hh, 16 hh + 16) and [32 + 16 hh, + 16) of the step's tile
-        const uint32_t d_lane = tmem_w + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(16 * hh);
+        const int lg = (32 * blk) / p.group;     // the block's group within the unit
+        const uint32_t coff = 2048u * (uint32_t)blk + 16u * (uint32_t)(n ^ (2 * blk));
+        const uint32_t soff = p.scales_off + 256u * (uint32_t)lg + 2u * (uint32_t)n;
+        const uint32_t zoff = p.zeros_off + 64u * (uint32_t)lg + 4u * (uint32_t)(n >> 3);
+        const int zsh = 4 * (n & 7);
+        // this warp's lanes of tensor memory (its 32 channels), columns [16 blk, 16 blk + 16) of the
+        // step's tile
+        const uint32_t d_lane = tmem_w + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(16 * blk);
         int rs = 0, s = 0;
         uint32_t rph = 0, ph = 0;
         bool ok = true;
@@ -384,42 +391,29 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             }
             for (int uu = 0; uu < nu; ++uu) {
                 const uint8_t* rec = ring_w + (size_t)rs * p.slot_w + (size_t)uu * R;
-                uint4 cw[2];
-                uint16_t sb[2];
-                uint32_t zv[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int blk = 2 * h + hh;
-                    cw[h] = *reinterpret_cast<const uint4*>(rec + 2048 * blk + 16 * (n ^ (2 * blk)));
-                    const int lg = (32 * blk) / group;
-                    sb[h] = *reinterpret_cast<const uint16_t*>(rec + p.scales_off + 256 * lg + 2 * n);
-                    zv[h] = sym ? 8u
-                                : (*reinterpret_cast<const uint32_t*>(rec + p.zeros_off + 64 * lg + 4 * (n >> 3)) >>
-                                   (4 * (n & 7))) & 0xFu;
-                }
+                const uint4 cw = *reinterpret_cast<const uint4*>(rec + coff);
+                const uint16_t sb = *reinterpret_cast<const uint16_t*>(rec + soff);
+                const uint32_t zv = sym ? 8u : (*reinterpret_cast<const uint32_t*>(rec + zoff) >> zsh) & 0xFu;
                 if (!tc_wait(&free_s[s], ph ^ 1u, abort_flag, p.dev_status, wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();   // the MMAs that read this tile completed before the stores
+                const uint32_t za = Ops::zz_a(zv), zb = Ops::zz_b(zv);
+                typename Ops::Scale sc;
+                sc.set(sb);
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint32_t out[16];   // column c: K pair (2 c, 2 c + 1) of the block
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t za = Ops::zz_a(zv[h]), zb = Ops::zz_b(zv[h]);
-                    typename Ops::Scale sc;
-                    sc.set(sb[h]);
-                    const uint32_t words[4] = {cw[h].x, cw[h].y, cw[h].z, cw[h].w};
-                    uint32_t out[16];   // column c: K pair (2 c, 2 c + 1) of the block
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        uint32_t r[4];
-                        Ops::unpack(words[w], km, r);
-                        out[4 * w + 0] = sc.apply(Ops::sub_a(r[0], za));
-                        out[4 * w + 1] = sc.apply(Ops::sub_b(r[1], zb));
-                        out[4 * w + 2] = sc.apply(Ops::sub_a(r[2], za));
-                        out[4 * w + 3] = sc.apply(Ops::sub_b(r[3], zb));
-                    }
-                    tmem_st16(d_lane + (uint32_t)(s * kTcStepCols + 32 * h), out);
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t r[4];
+                    Ops::unpack(words[w], km, r);
+                    out[4 * w + 0] = sc.apply(Ops::sub_a(r[0], za));
+                    out[4 * w + 1] = sc.apply(Ops::sub_b(r[1], zb));
+                    out[4 * w + 2] = sc.apply(Ops::sub_a(r[2], za));
+                    out[4 * w + 3] = sc.apply(Ops::sub_b(r[3], zb));
                 }
+                tmem_st16(d_lane + (uint32_t)(s * kTcStepCols), out);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
