@@ -231,8 +231,9 @@ W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);
 
 /*
  * w4a16_repack -- one-time load-time permutation of the plain packed layout into the tiled
- * layout that w4a16_gemm reads fastest. It is a bijection of bits: nothing is rounded or
- * re-quantized. "INT4 and Low-Bit Inference", section 5 "The kernel is half the story" (weights
+ * layout that w4a16_gemm reads fastest. The codes, zeros and scales are moved, not changed
+ * (except the scale of a group whose codes all equal its zero point, stored as 0): nothing is
+ * rounded or re-quantized, and every dequantized weight is the same. "INT4 and Low-Bit Inference", section 5 "The kernel is half the story" (weights
  * pre-permuted at load so unpacking is branch-free and coalesced); "4.3 Weight-only INT4",
  * section 4 (weights pre-reordered into a layout that suits runtime reads).
  * Tiled layout: one record per unit of 128 output channels x 128 input channels; unit (t, c)
@@ -243,6 +244,8 @@ W4A16_API size_t w4a16_repack_bytes(int K, int N, int group, int sym);
  *                     n % 128 owns the 16 bytes at slot ((n % 128) XOR 2h) of its block, and word
  *                     w (w = 0..3) of them is plain word (j, n) with j = 16 c + 4 h + w;
  *   then G x 256 B    scales: group row c * G + gg at 256 gg, channel n % 128 at + 2 (n % 128);
+ *                     a (group, channel) whose codes all equal its zero point (0 when symmetric)
+ *                     stores scale 0 -- its dequantized weights are 0 with either scale;
  *   then G x 64 B     zeros (asym only): group row c * G + gg at 64 gg, plain words
  *                     [16 t, 16 t + 16) of that row.
  * Each word is re-encoded: nibble slot p (bits 4p..4p+3, p = 0..3) holds the code of element 2p

@@ -340,7 +340,9 @@ int w4o_max_threads(void) {
  *     that of element 2p + 1 (element e = input channel 8 j + e); symmetric codes are stored
  *     offset-binary, q + 8 (zero-point 8);
  *   scales, from byte 8192: group gg (gg = 0..G-1, plain group row c * G + gg) at 8192 + 256 gg,
- *     channel n at + 2 n (fp16 bits);
+ *     channel n at + 2 n (fp16 bits), except that a (group, channel) whose codes all equal its
+ *     zero point (0 for the symmetric scheme) stores scale 0 (its dequantized weights are 0
+ *     with either scale);
  *   zeros (asymmetric only), from byte 8192 + 256 G: group gg at + 64 gg, the 16 plain words of
  *     the tile's channels (word n / 8 holds channel n at nibble n mod 8).
  * Records follow each other with no padding.
@@ -383,8 +385,15 @@ int w4o_repack(const int32_t* codes, const uint16_t* scales, const int32_t* zero
                     }
             for (long gg = 0; gg < G; ++gg) {
                 const long gi = c * G + gg;
-                for (long nl = 0; nl < 128; ++nl)
-                    memcpy(rec + off[2] + 256 * gg + 2 * nl, &scales[gi * N + 128 * t + nl], 2);
+                for (long nl = 0; nl < 128; ++nl) {
+                    const long n = 128 * t + nl;
+                    const uint32_t zp = sym ? 0u : ((uint32_t)zeros[gi * (N / 8) + n / 8] >> (4 * (n % 8))) & 0xFu;
+                    int all_zero_point = 1;
+                    for (long k = gi * group; k < (gi + 1) * group; ++k)
+                        if ((((uint32_t)codes[(k / 8) * N + n] >> (4 * (k % 8))) & 0xFu) != zp) all_zero_point = 0;
+                    const uint16_t sv = all_zero_point ? (uint16_t)0 : scales[gi * N + n];
+                    memcpy(rec + off[2] + 256 * gg + 2 * nl, &sv, 2);
+                }
                 if (!sym)
                     for (long wd = 0; wd < 16; ++wd)
                         memcpy(rec + off[4] + 64 * gg + 4 * wd, &zeros[gi * (N / 8) + 16 * t + wd], 4);

@@ -473,3 +473,30 @@ def test_tiled_layout_symmetric_is_offset_binary(oracle_mod):
     # word (j = 0, n = 0) sits at position 0: its slots hold q[0, 0..7 even], q[.. odd] + 8
     e = [q[k, 0] + 8 for k in range(8)]
     assert _slots(np.uint32(t[0])) == [e[0], e[2], e[4], e[6], e[1], e[3], e[5], e[7]]
+
+
+def test_tiled_layout_zero_point_groups_store_scale_zero(oracle_mod):
+    """A (group, channel) whose codes all equal its zero point -- the degenerate group, whose
+    dequantized weights are all zero -- stores scale 0 in the tiled buffer; every other scale is
+    copied. Dequantizing either buffer gives the same weights."""
+    K, N, group = 256, 128, 64
+    Wb = np.array(np.random.default_rng(5).standard_normal((K, N)) * 0.02, dtype=np.float16).view(np.uint16).copy()
+    Wb[64:128, 7] = 0                  # a group of zeros: scale rounds to 0, stored 1, codes = zero point
+    Wb[:64, 9] = 0x0001                # a sub-2^-25 range: the same
+    for sym in (0, 1):
+        st, codes, scales, zeros = oracle_mod.quantize(Wb, group, sym)
+        assert scales[1, 7] == 0x3C00 and scales[0, 9] == 0x3C00
+        buf = oracle_mod.repack(codes, scales, zeros, K, N, group, sym)
+        off = oracle_mod.tiled_offsets(K, N, group, sym)
+        G = 128 // group
+        recs = buf.reshape(-1, off["record"])
+        sc = np.concatenate([recs[c][8192: 8192 + G * 256].copy().view(np.uint16).reshape(G, 128)
+                             for c in range(K // 128)])          # tile 0: [K/g, 128]
+        expect = scales[:, :128].copy()
+        expect[1, 7] = 0
+        expect[0, 9] = 0
+        assert np.array_equal(sc, expect)
+        zeroed = scales.copy()
+        zeroed[1, 7] = zeroed[0, 9] = 0
+        assert np.array_equal(oracle_mod.dequant(codes, zeroed, zeros, K, N, group, sym),
+                              oracle_mod.dequant(codes, scales, zeros, K, N, group, sym))

@@ -89,7 +89,7 @@ struct GemvStreamPlan {
     bool ok;
     int ns;               // pipeline stages
     int ctas;             // persistent CTAs (one per SM)
-    size_t row_bytes, act_bytes, red_bytes, stage_bytes, smem;
+    size_t row_bytes, act_bytes, red_bytes, sa_bytes, stage_bytes, smem;
     size_t partial_bytes; // workspace after the counters (cut-tile sums, then the slices' outputs)
     int slices;           // launches over equal K slices (1: the whole K at once)
 };

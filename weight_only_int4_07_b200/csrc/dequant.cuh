@@ -11,6 +11,9 @@
 // (64 + z), (128 + u) - (128 + z). A scale s (an fp16 value) multiplies (u - z) with one
 // rounding: fp16 directly; bf16 as s = s_hi + s_lo with s_hi the bf16 truncation of s and s_lo
 // (at most 3 significant bits) exact in bf16, d s_lo exact, fma(d, s_hi, d s_lo) rounded once.
+// A third fp16 form needs no magic and no subtraction: the mask alone leaves u (or 16 u) in the
+// low mantissa bits of an fp16 whose exponent field is zero, the subnormal u 2^-24 (16 u 2^-24),
+// which the warp-level MMA multiplies exactly; the zero point then comes off the FP32 sums.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -77,6 +80,14 @@ struct GsOps<__half> {
             "{%0, %1, %2, %3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
             : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+    // the first MMA of a chain: C = 0
+    static __device__ __forceinline__ void mma_z(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%10, %10, %10, %10};"
+            : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
     }
 };
 

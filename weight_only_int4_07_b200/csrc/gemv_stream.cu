@@ -88,7 +88,7 @@ struct GsParams {
     int* dev_status;
     int M, K, N, sym, ns, P;
     uint32_t record, scales_off, zeros_off;
-    uint32_t stage_bytes, row_bytes, act_bytes, red_bytes;
+    uint32_t stage_bytes, row_bytes, act_bytes, red_bytes, sa_bytes;
     GsMasks km;
     GsMasks km_native;   // bf16 masks, for bf16 rows kept in bf16 at group 128
     // K slice of this launch: A points at its first column, rows lda elements apart; the slice's
@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
 
     uint8_t* acts = smem_raw;                                             // [M][RS]
     float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][groups - 1][M][128]
-    uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes;                 // 320 zero bytes
+    float* sa = reinterpret_cast<float*>(smem_raw + p.act_bytes + p.red_bytes);   // [K/128][Me] unit sums
+    uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes + p.sa_bytes;    // 320 zero bytes
     int* rowexp = reinterpret_cast<int*>(zrow + 320);                     // [16] largest exponent per row
     int* rowmin = reinterpret_cast<int*>(zrow + 384);                     // [16] smallest nonzero one
     uint8_t* stages = zrow + kGsZrowBytes;                                // ns x stage_bytes
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < 96; i += kGsThreads) reinterpret_cast<uint32_t*>(zrow)[i] = 0u;
+    if (threadIdx.x < 2) reinterpret_cast<uint32_t*>(zrow + 448)[threadIdx.x] = 0u;   // two zero sums
     if (threadIdx.x < 16) rowmin[threadIdx.x] = 255;
     __syncthreads();
     grid_dependents_launch();
@@ -256,6 +258,31 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     }
     __syncthreads();
 
+    // Group 128 on the fp16 arithmetic: the codes enter the MMAs as fp16 subnormals, so the zero
+    // point comes off the FP32 sums as z * sum_k a_k; those sums, one per row and unit (times
+    // 2^-24, the subnormals' scale), summed once per CTA from the staged activations in a fixed
+    // order: lane l of a warp adds four values of block l / 8 of the unit, then the warp's lanes.
+    constexpr bool kSub = kPost && std::is_same<MathT, __half>::value;
+    const int Me = (M + 1) & ~1;
+    if constexpr (kSub) {
+        if (!wide) {
+            for (int item = warp; item < M * steps; item += kGsWarps) {
+                const int m = item / steps, sp = item - m * steps;
+                const uint8_t* blk = acts + (uint32_t)m * RS + (uint32_t)sp * 320u + (uint32_t)(lane >> 3) * 80u +
+                                     (uint32_t)(lane & 7) * 8u;
+                const uint2 hv = *reinterpret_cast<const uint2*>(blk);
+                const __half2 h0 = *reinterpret_cast<const __half2*>(&hv.x), h1 = *reinterpret_cast<const __half2*>(&hv.y);
+                float v = (__low2float(h0) + __high2float(h0)) + (__low2float(h1) + __high2float(h1));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) sa[sp * Me + m] = v * 5.9604644775390625e-08f;   // 2^-24
+            }
+            if (M & 1)
+                for (int sp = threadIdx.x; sp < steps; sp += kGsThreads) sa[sp * Me + M] = 0.0f;
+            __syncthreads();
+        }
+    }
+
     // activation fragments: lane holds row 8 b + g (rows at or past M read a zero block)
     const uint8_t* abase[NB];
     uint32_t astride[NB];
@@ -264,6 +291,16 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         const bool real = 8 * b + g < M;
         abase[b] = real ? acts + (uint32_t)(8 * b + g) * RS + (uint32_t)t * 80u : zrow + (uint32_t)t * 80u;
         astride[b] = real ? 320u : 0u;
+    }
+
+    // unit sums of the two batch columns 8 b + 2 t, + 1 this lane's MMA results hold
+    const float* sbase[NB];
+    uint32_t sstride[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const bool real = 8 * b + 2 * t < M;
+        sbase[b] = real ? sa + 8 * b + 2 * t : reinterpret_cast<const float*>(zrow + 448);
+        sstride[b] = real ? (uint32_t)Me : 0u;
     }
 
     const GsMasks km = p.km;
@@ -481,6 +518,59 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         }
     };
 
+    // Group 128 on the fp16 arithmetic: each operand register is one AND of a packed word, which
+    // leaves the codes as fp16 subnormals u 2^-24 (pairs (0, 1), (4, 5) of the word) and 16 u 2^-24
+    // (pairs (2, 3), (6, 7)), multiplied exactly by the MMA and summed in two chains (lo, hi) per
+    // row tile; no magic exponent and no zero-point arithmetic per weight. Per unit and channel
+    // the zero point then comes off the FP32 sum, lo + hi / 16 - z sum_k a_k 2^-24, and the scale
+    // (times 2^24) multiplies the result. A group whose codes all equal its zero point has scale
+    // 0 in the tiled layout, so it adds exactly nothing.
+    auto unit_math_sub = [&](const uint4 (&cw)[4], const uint16_t (&sb)[4], const uint4& zw, const uint4 (&v)[NB][4],
+                             int sp) {
+        using O = GsOps<__half>;
+        const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+        float2 su[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) su[b] = *reinterpret_cast<const float2*>(sbase[b] + (uint32_t)sp * sstride[b]);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            // MMA rows g / g + 8: channels ch0 + 16 rt / ch0 + 16 rt + 8
+            const uint4 c0 = cw[2 * rt], c1 = cw[2 * rt + 1];
+            const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+            float alo[NB][4], ahi[NB][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t h0 = mulhi(w0[i], km.m8), h1 = mulhi(w1[i], km.m8);
+                const uint32_t a0 = w0[i] & 0x000F000Fu, a1 = w1[i] & 0x000F000Fu;
+                const uint32_t a2 = h0 & 0x000F000Fu, a3 = h1 & 0x000F000Fu;
+                const uint32_t b0 = w0[i] & 0x00F000F0u, b1 = w1[i] & 0x00F000F0u;
+                const uint32_t b2 = h0 & 0x00F000F0u, b3 = h1 & 0x00F000F0u;
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    if (i == 0) {
+                        O::mma_z(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
+                        O::mma_z(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
+                    } else {
+                        O::mma(alo[b], a0, a1, a2, a3, v[b][i].x, v[b][i].y);
+                        O::mma(ahi[b], b0, b1, b2, b3, v[b][i].z, v[b][i].w);
+                    }
+                }
+            }
+            const float z0 = (float)((zws[2 * rt] >> zsh) & 0xFu), z1 = (float)((zws[2 * rt + 1] >> zsh) & 0xFu);
+            const float s0 = __half2float(__ushort_as_half(sb[2 * rt])) * 16777216.0f;
+            const float s1 = __half2float(__ushort_as_half(sb[2 * rt + 1])) * 16777216.0f;
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                tot[rt][b][0] = fmaf(s0, fmaf(-z0, su[b].x, fmaf(ahi[b][0], 0.0625f, alo[b][0])), tot[rt][b][0]);
+                tot[rt][b][2] = fmaf(s1, fmaf(-z1, su[b].x, fmaf(ahi[b][2], 0.0625f, alo[b][2])), tot[rt][b][2]);
+                if (ODD) {
+                    tot[rt][b][1] = fmaf(s0, fmaf(-z0, su[b].y, fmaf(ahi[b][1], 0.0625f, alo[b][1])), tot[rt][b][1]);
+                    tot[rt][b][3] = fmaf(s1, fmaf(-z1, su[b].y, fmaf(ahi[b][3], 0.0625f, alo[b][3])), tot[rt][b][3]);
+                }
+            }
+        }
+    };
+
     bool aborted = false;
     int s_idx = -1;
     uint32_t ph = 0;
@@ -529,7 +619,9 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         }
         if constexpr (kConv) {
             if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
-            else unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
+            else unit_math_sub(cw, sb, zw, v, sp);
+        } else if constexpr (kSub) {
+            unit_math_sub(cw, sb, zw, v, sp);
         } else {
             unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
         }
@@ -623,9 +715,10 @@ GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
     pl.row_bytes = 320 * units + ((units & 1) ? 0 : 64);          // 80-byte blocks; rows 64 mod 128 apart
     pl.act_bytes = ((size_t)M * pl.row_bytes + 127) & ~(size_t)127;
     pl.red_bytes = (size_t)2 * (kGsGroups - 1) * M * 128 * 4;
+    pl.sa_bytes = (((size_t)units * ((M + 1) & ~1) * 4) + 127) & ~(size_t)127;   // unit sums (group 128)
     pl.stage_bytes = ((size_t)kGsUnitsPerStage * L.record + 127) & ~(size_t)127;
     const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 8 + 8 * kGsMaxStages + 127) & ~(size_t)127;
-    const size_t fixed = pl.act_bytes + pl.red_bytes + kGsZrowBytes + flags;
+    const size_t fixed = pl.act_bytes + pl.red_bytes + pl.sa_bytes + kGsZrowBytes + flags;
     if (fixed >= (size_t)kGsSmemMax) return pl;
     size_t ns = ((size_t)kGsSmemMax - fixed) / pl.stage_bytes;
     if (ns > kGsMaxStages) ns = kGsMaxStages;
@@ -691,6 +784,7 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.row_bytes = (uint32_t)pl.row_bytes;
     prm.act_bytes = (uint32_t)pl.act_bytes;
     prm.red_bytes = (uint32_t)pl.red_bytes;
+    prm.sa_bytes = (uint32_t)pl.sa_bytes;
     prm.lda = K;
     prm.ktot = K / 128;
     prm.wait_ns = wait_limit_ns();
