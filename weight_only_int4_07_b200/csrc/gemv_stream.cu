@@ -14,12 +14,13 @@
 // of its range, waits for the count (acquire, bounded), adds the sums in CTA order, writes C and
 // resets the counter. The result does not depend on timing.
 //
-// Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each;
-// lane 0 of each warp leaving a stage counts the warp out on a shared counter, and the warp that
-// completes the count refills the slot with the stage ns positions later, so no warp waits for
-// another to issue a copy. Sixteen warps in four groups: group q takes unit q of every stage,
-// warp w of a group owns channels 32 w .. 32 w + 31 of the unit. At the end of a tile group 0
-// adds the four groups' sums (handed over through shared memory and one CTA barrier).
+// Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each.
+// Sixteen compute warps in four groups: group q takes unit q of every stage, warp w of a group
+// owns channels 32 w .. 32 w + 31 of the unit; leaving a stage, each warp arrives on the slot's
+// `empty` barrier. Two service warps: a producer warp refills a slot with the stage ns positions
+// later once all sixteen have left it, and an epilogue warp adds the four groups' sums of each
+// tile (handed over through shared memory and an mbarrier) and writes C or runs the cut-tile
+// protocol. No compute warp waits for another: they wait only for their data.
 //
 // Math (warp-level tensor-core MMA, m16n8k16, FP32 accumulators), per warp and unit: lane
 // (g = lane / 4, t = lane % 4) reads the 16 bytes of block t (32 K) of channels 32 w + g + 8 r,
@@ -52,9 +53,11 @@ using namespace sm100;
 // Four groups of 4 warps per CTA (each group takes one unit of a stage), one CTA per SM. (Two
 // groups and two CTAs per SM, which let the next launch's CTAs start on an SM before the previous
 // launch has left it, measured 12% slower on the Llama-3-70B-shaped stack.)
-constexpr int kGsGroups = 4, kGsGroupWarps = 4, kGsWarps = kGsGroups * kGsGroupWarps;
+constexpr int kGsGroups = 4, kGsGroupWarps = 4, kGsWarps = kGsGroups * kGsGroupWarps;   // compute warps
 constexpr int kGsCtasPerSm = 1;
-constexpr int kGsThreads = 32 * kGsWarps;
+// two service warps after the compute warps: one issues the weight copies, one sums the tiles
+constexpr int kGsWarpProducer = kGsWarps, kGsWarpEpilogue = kGsWarps + 1, kGsAllWarps = kGsWarps + 2;
+constexpr int kGsThreads = 32 * kGsAllWarps;
 constexpr int kGsUnitsPerStage = kGsGroups;
 static_assert(kGsGroups >= 2 && kGsGroups <= 4, "two to four groups");
 constexpr int kGsMinStages = 3, kGsMaxStages = 16;
@@ -62,9 +65,6 @@ constexpr int kGsSmemMax = (228 * 1024) / kGsCtasPerSm - 1024;   // per CTA; 1 K
 constexpr uint64_t kGsSpin = 2000000000ull;
 constexpr int kGsZrowBytes = 512;   // the zero activation block, then per-row exponent bounds
 
-__device__ __forceinline__ void named_bar(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
@@ -125,23 +125,29 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const uint32_t R = p.record, stage_bytes = p.stage_bytes, RS = p.row_bytes;
 
     uint8_t* acts = smem_raw;                                             // [M][RS]
-    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][groups - 1][M][128]
+    float* red = reinterpret_cast<float*>(smem_raw + p.act_bytes);        // [2][groups][M][128]
     float* sa = reinterpret_cast<float*>(smem_raw + p.act_bytes + p.red_bytes);   // [K/128][Me] unit sums
     uint8_t* zrow = smem_raw + p.act_bytes + p.red_bytes + p.sa_bytes;    // 320 zero bytes
     int* rowexp = reinterpret_cast<int*>(zrow + 320);                     // [16] largest exponent per row
     int* rowmin = reinterpret_cast<int*>(zrow + 384);                     // [16] smallest nonzero one
     uint8_t* stages = zrow + kGsZrowBytes;                                // ns x stage_bytes
-    uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);
-    int* flags = reinterpret_cast<int*>(full + ns);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)ns * stage_bytes);   // [ns] stage landed
+    uint64_t* empty = full + ns;        // [ns] the 16 compute warps left the slot's stage
+    uint64_t* tfull = empty + ns;       // [2] the groups' sums of a tile are in `red`
+    uint64_t* tempty = tfull + 2;       // [2] the epilogue warp has read them
+    int* flags = reinterpret_cast<int*>(tempty + 2);
     volatile int* abort_flag = flags;
     int* issued = flags + 2;            // [ns] copies issued into each slot
-    int* leave = flags + 2 + ns;        // [ns] warps that have left the slot's current stage
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kGsWarps);
             issued[i] = 0;
-            leave[i] = 0;
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], kGsWarps);
+            mbar_init(&tempty[i], 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -174,9 +180,10 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                 bulk_g2s(dst + (size_t)n1 * R, p.tiled + ((size_t)(t + 1) * p.ktot + p.c0) * R, (uint32_t)(n - n1) * R,
                          &full[s]);
         }
-        atomicAdd(&issued[s], 1);
+        ++issued[s];
     };
-    if (threadIdx.x == 0)
+    const bool producer = warp == kGsWarpProducer && lane == 0;
+    if (producer)
         for (int st = 0; st < nst && st < ns; ++st) issue(st);
 
     const int grp = warp / kGsGroupWarps, wg = warp % kGsGroupWarps;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const int Me = (M + 1) & ~1;
     if constexpr (kSub) {
         if (!wide) {
-            for (int item = warp; item < M * steps; item += kGsWarps) {
+            for (int item = warp; item < M * steps; item += kGsAllWarps) {
                 const int m = item / steps, sp = item - m * steps;
                 const uint8_t* blk = acts + (uint32_t)m * RS + (uint32_t)sp * 320u + (uint32_t)(lane >> 3) * 80u +
                                      (uint32_t)(lane & 7) * 8u;
@@ -324,130 +331,30 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     int seg_lo = 0, sp_lo = (int)(u0 - (long long)tile * steps);
     int seg_hi = (steps - sp_lo) < nunits ? (steps - sp_lo) : nunits;
 
-    // end of a tile segment: groups 1..3 hand their sums to group 0 through shared memory (two
-    // buffers, by tile parity, so one CTA barrier per tile suffices); group 0 writes C, or this
-    // CTA's partial sums when the tile is cut between CTAs. (A variant without the CTA barrier,
-    // the summing group rotating over tiles and the others handing over through mbarriers and
-    // going on, measured 1.5% slower on the Llama-3-70B-shaped stack.)
-    auto emit = [&]() {
-        float* rb = red + (size_t)(tile & 1) * (kGsGroups - 1) * M * 128;
-        if (grp > 0) {
+    // End of a tile segment (compute warps): each group writes its FP32 sums of the tile's 128
+    // channels to one of two shared buffers (by tile parity) and arrives on its `full` barrier; the
+    // epilogue warp adds the four groups' sums and writes C (or this CTA's partial sums when the
+    // tile is cut between CTAs) and frees the buffer. A group waits only before it reuses a buffer
+    // two tiles later, which the epilogue warp has normally long released; no compute warp waits
+    // for another.
+    int n_tile = 0;
+    auto tile_end = [&]() {
+        const int bsel = n_tile & 1;
+        const uint32_t use = (uint32_t)(n_tile >> 1) & 1u;
+        (void)wait_uniform(&tempty[bsel], use ^ 1u, abort_flag, p.dev_status, p.wait_ns);
+        float* rb = red + ((size_t)bsel * kGsGroups + grp) * M * 128;
 #pragma unroll
-            for (int rt = 0; rt < 2; ++rt)
+        for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-                for (int b = 0; b < NB; ++b)
+            for (int b = 0; b < NB; ++b)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                        if (m < M) rb[((grp - 1) * M + m) * 128 + ch] = tot[rt][b][e];
-                    }
-        }
-        __syncthreads();
-        if (grp == 0) {
-            T* C = static_cast<T*>(p.C);
-            const size_t n0 = (size_t)tile * 128;
-            const int cf = unit_owner((long long)tile * steps, U, P);
-            const int cl = unit_owner((long long)tile * steps + steps - 1, U, P);
-            float vals[2][NB][4];
-#pragma unroll
-            for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                        float v = tot[rt][b][e];
-#pragma unroll
-                        for (int j = 0; j < kGsGroups - 1; ++j) v += m < M ? rb[(j * M + m) * 128 + ch] : 0.0f;
-                        vals[rt][b][e] = m < M ? v : 0.0f;
-                    }
-            const bool first = threadIdx.x == 0;
-            if (cf == cl || cta == cf) {
-                if (cf != cl) {
-                    // the tile is cut between CTAs cf .. cl and this is cf: the tile is the last of
-                    // its range. Wait until every later CTA of the tile has published its sums (they
-                    // hold the tile at the start of their ranges), then add them in CTA order.
-                    if (first) {
-                        const uint64_t t0 = globaltimer_ns();
-                        for (;;) {
-                            int n;
-                            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + tile)
-                                         : "memory");
-                            if (n >= cl - cf) break;
-                            if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
-                                *abort_flag = 1;
-                                report_status(p.dev_status, W4A16_ETIMEOUT);
-                                break;
-                            }
-                        }
-                        p.counters[tile] = 0;
-                    }
-                    named_bar(2, 32 * kGsGroupWarps);
-                    // the loads of up to kPL contributors are in flight together; the sums are
-                    // added in CTA order
-                    constexpr int kPL = NB == 1 ? 4 : 2;
-                    for (int c0 = cf + 1; c0 <= cl; c0 += kPL) {
-                        float ld[kPL][2][NB][4];
-#pragma unroll
-                        for (int j = 0; j < kPL; ++j) {
-                            const float* part = p.partials + (size_t)(c0 + j) * M * 128;
-#pragma unroll
-                            for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                                for (int b = 0; b < NB; ++b)
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                                        ld[j][rt][b][e] = (m < M && c0 + j <= cl) ? __ldcg(part + m * 128 + ch) : 0.0f;
-                                    }
-                        }
-#pragma unroll
-                        for (int j = 0; j < kPL; ++j)
-#pragma unroll
-                            for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                                for (int b = 0; b < NB; ++b)
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e)
-                                        if (c0 + j <= cl) vals[rt][b][e] += ld[j][rt][b][e];
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
+                    if (m < M) rb[m * 128 + ch] = tot[rt][b][e];
                 }
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                            if (m < M) {
-                                float y = vals[rt][b][e];
-                                if constexpr (kConv)   // undo the row's 2^-k
-                                    if (!wide) y *= __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
-                                if (p.out_f32)
-                                    p.out_f32[(size_t)m * N + n0 + ch] = y;
-                                else
-                                    C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(y);
-                            }
-                        }
-            } else {
-                // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
-                // count them, without waiting
-                float* part = p.partials + (size_t)cta * M * 128;
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int m = 8 * b + 2 * t + (e & 1), ch = ch0 + 16 * rt + 8 * (e >> 1);
-                            if (m < M) part[m * 128 + ch] = vals[rt][b][e];
-                        }
-                __threadfence();
-                named_bar(2, 32 * kGsGroupWarps);
-                if (first)
-                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + tile) : "memory");
-            }
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[bsel]);
+        ++n_tile;
         zero_tot();
         ++tile;
         sp_lo = 0;
@@ -571,69 +478,165 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         }
     };
 
-    bool aborted = false;
-    int s_idx = -1;
-    uint32_t ph = 0;
-    for (int st = 0; st < nst; ++st) {
-        if (st > 0 && !aborted) {
-            // leave stage st - 1: every read of the slot by this warp has completed (its values
-            // were consumed by the unit's MMAs), so lane 0 counts the warp out once; the warp
-            // that completes the count of 16 refills the slot with stage st - 1 + ns. No warp
-            // waits for another.
-            __syncwarp();
-            if (lane == 0) {
-                int old;
-                asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
-                             : "=r"(old) : "r"(smem_u32(&leave[s_idx])) : "memory");
-                if (old == kGsWarps - 1) {
-                    leave[s_idx] = 0;
-                    if (st - 1 + ns < nst) issue(st - 1 + ns);
-                }
+    if (warp == kGsWarpProducer) {
+        // ------------------------------------------------------------ producer (lane 0)
+        // refills slot s with stage st once the 16 compute warps have left stage st - ns
+        if (lane == 0) {
+            for (int st = ns; st < nst; ++st) {
+                if (!mbar_wait(&empty[st % ns], (uint32_t)((st / ns) - 1) & 1u, abort_flag, p.dev_status, p.wait_ns))
+                    break;
+                issue(st);
             }
         }
-        if (++s_idx == ns) {
-            s_idx = 0;
-            ph ^= 1u;
+    } else if (warp == kGsWarpEpilogue) {
+        // ------------------------------------------------------------ epilogue warp
+        // per tile segment of this CTA's range: the four groups' sums (in group order), then C, or
+        // the cut-tile protocol; lane l handles channels l + 32 j
+        T* C = static_cast<T*>(p.C);
+        int etile = (int)(u0 / steps);
+        int elo = 0;
+        int ehi = (steps - (int)(u0 - (long long)etile * steps)) < nunits ? (steps - (int)(u0 - (long long)etile * steps))
+                                                                            : nunits;
+        for (int et = 0; elo < nunits; ++et) {
+            const int bsel = et & 1;
+            (void)wait_uniform(&tfull[bsel], (uint32_t)(et >> 1) & 1u, abort_flag, p.dev_status, p.wait_ns);
+            const float* rb = red + (size_t)bsel * kGsGroups * M * 128;
+            const size_t n0 = (size_t)etile * 128;
+            const int cf = unit_owner((long long)etile * steps, U, P);
+            const int cl = unit_owner((long long)etile * steps + steps - 1, U, P);
+            if (cf == cl || cta == cf) {
+                if (cf != cl) {
+                    // the tile is cut between CTAs cf .. cl and this is cf: the tile is the last of
+                    // its range. Wait until every later CTA of the tile has published its sums (they
+                    // hold the tile at the start of their ranges), then add them in CTA order.
+                    if (lane == 0) {
+                        const uint64_t t0 = globaltimer_ns();
+                        for (;;) {
+                            int n;
+                            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + etile)
+                                         : "memory");
+                            if (n >= cl - cf) break;
+                            if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+                                *abort_flag = 1;
+                                report_status(p.dev_status, W4A16_ETIMEOUT);
+                                break;
+                            }
+                        }
+                        p.counters[etile] = 0;
+                    }
+                    __syncwarp();
+                }
+                for (int m = 0; m < M; ++m) {
+                    float up = 1.0f;
+                    if constexpr (kConv)   // undo the row's 2^-k
+                        if (!wide) up = __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
+                    float y[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int ch = lane + 32 * j;
+                        y[j] = rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
+                               rb[(3 * M + m) * 128 + ch];
+                    }
+                    // the later CTAs' sums, in CTA order; the loads of four CTAs in flight together
+                    for (int c0 = cf + 1; cf != cl && c0 <= cl; c0 += 4) {
+                        float ld[4][4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                ld[q][j] = c0 + q <= cl ? __ldcg(p.partials + ((size_t)(c0 + q) * M + m) * 128 + lane + 32 * j)
+                                                        : 0.0f;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (c0 + q <= cl) y[j] += ld[q][j];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int ch = lane + 32 * j;
+                        const float o = y[j] * up;
+                        if (p.out_f32)
+                            p.out_f32[(size_t)m * N + n0 + ch] = o;
+                        else
+                            C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(o);
+                    }
+                }
+            } else {
+                // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
+                // count them, without waiting
+                float* part = p.partials + (size_t)cta * M * 128;
+                for (int m = 0; m < M; ++m)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int ch = lane + 32 * j;
+                        part[m * 128 + ch] = rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] +
+                                             rb[(2 * M + m) * 128 + ch] + rb[(3 * M + m) * 128 + ch];
+                    }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0)
+                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + etile) : "memory");
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[bsel]);
+            ++etile;
+            elo = ehi;
+            ehi = elo + steps < nunits ? elo + steps : nunits;
         }
-        if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status, p.wait_ns)) aborted = true;
-        const int li = st * kGsUnitsPerStage + grp;
-        if (li >= nunits) continue;
-        while (li >= seg_hi) emit();
-        if (aborted) continue;
-        const int sp = sp_lo + (li - seg_lo);
-        const uint8_t* rec = stages + (uint32_t)s_idx * stage_bytes + rec_off;
-        uint4 cw[4];
+    } else {
+        // ------------------------------------------------------------ compute warps
+        bool aborted = false;
+        int s_idx = -1;
+        uint32_t ph = 0;
+        for (int st = 0; st < nst; ++st) {
+            if (++s_idx == ns) {
+                s_idx = 0;
+                ph ^= 1u;
+            }
+            if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status, p.wait_ns)) aborted = true;
+            const int li = st * kGsUnitsPerStage + grp;
+            if (li < nunits) {
+                while (li >= seg_hi) tile_end();
+                if (!aborted) {
+                    const int sp = sp_lo + (li - seg_lo);
+                    const uint8_t* rec = stages + (uint32_t)s_idx * stage_bytes + rec_off;
+                    uint4 cw[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) cw[r] = *reinterpret_cast<const uint4*>(rec + coff + 128 * r);
-        uint16_t sb[4];
+                    for (int r = 0; r < 4; ++r) cw[r] = *reinterpret_cast<const uint4*>(rec + coff + 128 * r);
+                    uint16_t sb[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) sb[r] = *reinterpret_cast<const uint16_t*>(rec + soff + 16 * r);
-        uint4 zw = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);   // symmetric: z = 8
-        if (!sym) zw = *reinterpret_cast<const uint4*>(rec + zoff);
-        uint4 v[NB][4];
+                    for (int r = 0; r < 4; ++r) sb[r] = *reinterpret_cast<const uint16_t*>(rec + soff + 16 * r);
+                    uint4 zw = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);   // symmetric: z = 8
+                    if (!sym) zw = *reinterpret_cast<const uint4*>(rec + zoff);
+                    uint4 v[NB][4];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const uint8_t* a = abase[b] + (uint32_t)sp * astride[b];
+                    for (int b = 0; b < NB; ++b) {
+                        const uint8_t* a = abase[b] + (uint32_t)sp * astride[b];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[b][i] = *reinterpret_cast<const uint4*>(a + 16 * i);
+                        for (int i = 0; i < 4; ++i) v[b][i] = *reinterpret_cast<const uint4*>(a + 16 * i);
+                    }
+                    if constexpr (kConv) {
+                        if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
+                        else unit_math_sub(cw, sb, zw, v, sp);
+                    } else if constexpr (kSub) {
+                        unit_math_sub(cw, sb, zw, v, sp);
+                    } else {
+                        unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
+                    }
+                }
+            }
+            // leave the stage: this warp's reads of the slot were consumed by its MMAs
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s_idx]);
         }
-        if constexpr (kConv) {
-            if (wide) unit_math(OpsTag<GsOps<__nv_bfloat16>>{}, p.km_native, cw, sb, zw, v);
-            else unit_math_sub(cw, sb, zw, v, sp);
-        } else if constexpr (kSub) {
-            unit_math_sub(cw, sb, zw, v, sp);
-        } else {
-            unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
-        }
+        while (seg_lo < nunits) tile_end();
     }
-    while (seg_lo < nunits) emit();
 
-    // after a timeout: let every copy still in flight land before the CTA exits (a wait that
-    // does not give up on the raised abort flag, still bounded in time). The barrier first: a warp
-    // that completes the count-out of a stage issues its refill, so the copies issued are known
-    // only once every warp has left the loop.
+    // after a timeout: let every copy still in flight land before the CTA exits (a wait that does
+    // not give up on the raised abort flag, still bounded in time); only the producer issues copies
     __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) {
+    if (producer && *abort_flag) {
         volatile int keep_waiting = 0;
         for (int s = 0; s < ns; ++s)
             if (issued[s] > 0) mbar_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u, &keep_waiting, nullptr, kGsSpin);
@@ -714,10 +717,10 @@ GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
     const size_t units = (size_t)(Ks / 128);
     pl.row_bytes = 320 * units + ((units & 1) ? 0 : 64);          // 80-byte blocks; rows 64 mod 128 apart
     pl.act_bytes = ((size_t)M * pl.row_bytes + 127) & ~(size_t)127;
-    pl.red_bytes = (size_t)2 * (kGsGroups - 1) * M * 128 * 4;
+    pl.red_bytes = (size_t)2 * kGsGroups * M * 128 * 4;
     pl.sa_bytes = (((size_t)units * ((M + 1) & ~1) * 4) + 127) & ~(size_t)127;   // unit sums (group 128)
     pl.stage_bytes = ((size_t)kGsUnitsPerStage * L.record + 127) & ~(size_t)127;
-    const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 8 + 8 * kGsMaxStages + 127) & ~(size_t)127;
+    const size_t flags = ((size_t)2 * kGsMaxStages * 8 + 32 + 8 + 4 * kGsMaxStages + 127) & ~(size_t)127;
     const size_t fixed = pl.act_bytes + pl.red_bytes + pl.sa_bytes + kGsZrowBytes + flags;
     if (fixed >= (size_t)kGsSmemMax) return pl;
     size_t ns = ((size_t)kGsSmemMax - fixed) / pl.stage_bytes;
