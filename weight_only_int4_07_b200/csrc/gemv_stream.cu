@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     // significant bits, so the conversion is exact; the MMAs then form the same products
     // a * (u - z) as bf16 operands would, and the sums are multiplied back by 2^k when C is
     // written. When some row holds a nonzero value further below its maximum, every CTA keeps
-    // the bf16 values and the bf16 arithmetic (the decision depends only on A, so all CTAs agree).
+    // the bf16 values and the bf16 arithmetic. Each CTA decides from the part of A it stages and
+    // takes its own sums back to the scale of A before they leave it, so CTAs need not agree.
     constexpr bool kConv = kPost && std::is_same<T, __nv_bfloat16>::value;
     using MathT = typename std::conditional<kConv, __half, T>::type;
     using Ops = GsOps<MathT>;
@@ -193,30 +194,38 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
 
     bool wide = false;   // kConv: some row keeps bf16 values and the bf16 arithmetic
 
+    // The units of K this CTA's range touches: all of them when the range holds a whole tile, else
+    // a run of nneed units from sp0, wrapping at the end of the tile. Only their activations are
+    // staged, scanned and summed (a CTA of the 28672-input down projection touches 43% of K).
+    const int sp0 = (int)(u0 % steps);
+    const int nneed = nunits < steps ? nunits : steps;
+    const int nchunk = 16 * nneed;   // 8-element chunks of A
+    auto need_chunk = [&](int q) { return 16 * ((sp0 + (q >> 4)) % steps) + (q & 15); };
+
     // A may be the output of the previous kernel in the stream
     grid_dependency_wait();
     {
         // activations: 32-K block t of unit sp at sp * 320 + 80 t (the 16-byte padding makes the
         // lanes' 16-byte reads conflict free); pairs in each 16-byte chunk stored (p0, p2, p1, p3)
         // so that each MMA's two B registers are adjacent; each CTA starts at a different chunk
-        const int vpr = K / 8;
+        const int rot = (cta * 64) % nchunk;
         auto chunk_off = [&](int m, int c) {
             return (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u + (uint32_t)((c >> 2) & 3) * 80u +
                    (uint32_t)(c & 3) * 16u;
         };
         for (int m = 0; m < M; ++m) {
             uint32_t emax = 0, emin = 255;   // largest, smallest nonzero biased exponent of row m
-            for (int c0 = threadIdx.x; c0 < vpr; c0 += 4 * kGsThreads) {
+            for (int c0 = threadIdx.x; c0 < nchunk; c0 += 4 * kGsThreads) {
                 uint4 vv[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    if (c0 + j * kGsThreads < vpr)
-                        vv[j] = *reinterpret_cast<const uint4*>(A + (size_t)m * p.lda +
-                                                                 8 * ((c0 + j * kGsThreads + cta * 64) % vpr));
+                    if (c0 + j * kGsThreads < nchunk)
+                        vv[j] = *reinterpret_cast<const uint4*>(
+                            A + (size_t)m * p.lda + 8 * need_chunk((c0 + j * kGsThreads + rot) % nchunk));
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    if (c0 + j * kGsThreads < vpr) {
-                        const int c = (c0 + j * kGsThreads + cta * 64) % vpr;
+                    if (c0 + j * kGsThreads < nchunk) {
+                        const int c = need_chunk((c0 + j * kGsThreads + rot) % nchunk);
                         *reinterpret_cast<uint4*>(acts + chunk_off(m, c)) =
                             make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
                         if constexpr (kConv) {
@@ -247,8 +256,8 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
             for (int m = 0; m < M && !wide; ++m) {
                 const int k = min(max(rowexp[m] - 141, -100), 114);
                 const float down = __int_as_float((127 - k) << 23);
-                for (int c0 = threadIdx.x; c0 < vpr; c0 += kGsThreads) {
-                    const int c = (c0 + cta * 64) % vpr;
+                for (int c0 = threadIdx.x; c0 < nchunk; c0 += kGsThreads) {
+                    const int c = need_chunk((c0 + rot) % nchunk);
                     uint4* q = reinterpret_cast<uint4*>(acts + chunk_off(m, c));
                     uint4 v = *q;
                     uint32_t* w = reinterpret_cast<uint32_t*>(&v);
@@ -273,8 +282,8 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const int Me = (M + 1) & ~1;
     if constexpr (kSub) {
         if (!wide) {
-            for (int item = warp; item < M * steps; item += kGsAllWarps) {
-                const int m = item / steps, sp = item - m * steps;
+            for (int item = warp; item < M * nneed; item += kGsAllWarps) {
+                const int m = item / nneed, sp = (sp0 + item - m * nneed) % steps;
                 const uint8_t* blk = acts + (uint32_t)m * RS + (uint32_t)sp * 320u + (uint32_t)(lane >> 3) * 80u +
                                      (uint32_t)(lane & 7) * 8u;
                 const uint2 hv = *reinterpret_cast<const uint2*>(blk);
@@ -285,7 +294,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                 if (lane == 0) sa[sp * Me + m] = v * 5.9604644775390625e-08f;   // 2^-24
             }
             if (M & 1)
-                for (int sp = threadIdx.x; sp < steps; sp += kGsThreads) sa[sp * Me + M] = 0.0f;
+                for (int q = threadIdx.x; q < nneed; q += kGsThreads) sa[((sp0 + q) % steps) * Me + M] = 0.0f;
             __syncthreads();
         }
     }
@@ -530,12 +539,12 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                     float up = 1.0f;
                     if constexpr (kConv)   // undo the row's 2^-k
                         if (!wide) up = __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
-                    float y[4];
+                    float y[4];   // this CTA's sums, back in the scale of A
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int ch = lane + 32 * j;
-                        y[j] = rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
-                               rb[(3 * M + m) * 128 + ch];
+                        y[j] = (rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
+                                rb[(3 * M + m) * 128 + ch]) * up;
                     }
                     // the later CTAs' sums, in CTA order; the loads of four CTAs in flight together
                     for (int c0 = cf + 1; cf != cl && c0 <= cl; c0 += 4) {
@@ -555,7 +564,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int ch = lane + 32 * j;
-                        const float o = y[j] * up;
+                        const float o = y[j];
                         if (p.out_f32)
                             p.out_f32[(size_t)m * N + n0 + ch] = o;
                         else
@@ -566,13 +575,17 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                 // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
                 // count them, without waiting
                 float* part = p.partials + (size_t)cta * M * 128;
-                for (int m = 0; m < M; ++m)
+                for (int m = 0; m < M; ++m) {
+                    float up = 1.0f;
+                    if constexpr (kConv)   // undo the row's 2^-k (this CTA's)
+                        if (!wide) up = __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int ch = lane + 32 * j;
-                        part[m * 128 + ch] = rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] +
-                                             rb[(2 * M + m) * 128 + ch] + rb[(3 * M + m) * 128 + ch];
+                        part[m * 128 + ch] = (rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] +
+                                              rb[(2 * M + m) * 128 + ch] + rb[(3 * M + m) * 128 + ch]) * up;
                     }
+                }
                 __threadfence();
                 __syncwarp();
                 if (lane == 0)
