@@ -200,104 +200,122 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const int sp0 = (int)(u0 % steps);
     const int nneed = nunits < steps ? nunits : steps;
     const int nchunk = 16 * nneed;   // 8-element chunks of A
-    auto need_chunk = [&](int q) { return 16 * ((sp0 + (q >> 4)) % steps) + (q & 15); };
 
     // A may be the output of the previous kernel in the stream
     grid_dependency_wait();
-    {
-        // activations: 32-K block t of unit sp at sp * 320 + 80 t (the 16-byte padding makes the
-        // lanes' 16-byte reads conflict free); pairs in each 16-byte chunk stored (p0, p2, p1, p3)
-        // so that each MMA's two B registers are adjacent; each CTA starts at a different chunk
-        const int rot = (cta * 64) % nchunk;
-        auto chunk_off = [&](int m, int c) {
-            return (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u + (uint32_t)((c >> 2) & 3) * 80u +
-                   (uint32_t)(c & 3) * 16u;
-        };
-        for (int m = 0; m < M; ++m) {
-            uint32_t emax = 0, emin = 255;   // largest, smallest nonzero biased exponent of row m
-            for (int c0 = threadIdx.x; c0 < nchunk; c0 += 4 * kGsThreads) {
-                uint4 vv[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (c0 + j * kGsThreads < nchunk)
-                        vv[j] = *reinterpret_cast<const uint4*>(
-                            A + (size_t)m * p.lda + 8 * need_chunk((c0 + j * kGsThreads + rot) % nchunk));
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (c0 + j * kGsThreads < nchunk) {
-                        const int c = need_chunk((c0 + j * kGsThreads + rot) % nchunk);
-                        *reinterpret_cast<uint4*>(acts + chunk_off(m, c)) =
-                            make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
-                        if constexpr (kConv) {
-                            const uint32_t x[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const uint32_t e0 = (x[q] >> 7) & 0xFFu, e1 = (x[q] >> 23) & 0xFFu;
-                                emax = max(emax, max(e0, e1));
-                                if (x[q] & 0x7FFFu) emin = min(emin, e0);
-                                if (x[q] & 0x7FFF0000u) emin = min(emin, e1);
-                            }
-                        }
-                    }
-            }
-            if constexpr (kConv) {
-                emax = __reduce_max_sync(0xffffffffu, emax);
-                emin = __reduce_min_sync(0xffffffffu, emin);
-                if (lane == 0) {
-                    atomicMax(&rowexp[m], (int)emax);
-                    atomicMin(&rowmin[m], (int)emin);
-                }
-            }
-        }
-        if constexpr (kConv) {
-            // second pass, in shared memory: bf16 -> 2^-k * a in fp16, unless some row is too wide
-            __syncthreads();
-            for (int m = 0; m < M; ++m) wide = wide || rowexp[m] - rowmin[m] > 31;
-            for (int m = 0; m < M && !wide; ++m) {
-                const int k = min(max(rowexp[m] - 141, -100), 114);
-                const float down = __int_as_float((127 - k) << 23);
-                for (int c0 = threadIdx.x; c0 < nchunk; c0 += kGsThreads) {
-                    const int c = need_chunk((c0 + rot) % nchunk);
-                    uint4* q = reinterpret_cast<uint4*>(acts + chunk_off(m, c));
-                    uint4 v = *q;
-                    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16) * down,
-                                                      __uint_as_float(w[i] & 0xFFFF0000u) * down);
-                        w[i] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                    *q = v;
-                }
-            }
-        }
-    }
-    __syncthreads();
 
-    // Group 128 on the fp16 arithmetic: the codes enter the MMAs as fp16 subnormals, so the zero
-    // point comes off the FP32 sums as z * sum_k a_k; those sums, one per row and unit (times
-    // 2^-24, the subnormals' scale), summed once per CTA from the staged activations in a fixed
-    // order: lane l of a warp adds four values of block l / 8 of the unit, then the warp's lanes.
+    // Staging: activations: 32-K block t of unit sp at sp * 320 + 80 t (the 16-byte padding makes
+    // the lanes' 16-byte reads conflict free); pairs in each 16-byte chunk stored (p0, p2, p1, p3)
+    // so that each MMA's two B registers are adjacent; each CTA starts at a different chunk. Chunk
+    // c0 of the pass (c0 = thread + i * threads) is chunk q = c0 + rot (mod nchunk) of the needed
+    // run; since threads, rot and nchunk are multiples of 16, the 16 lanes of a half warp hold the
+    // 16 chunks of one unit, whose sum (group 128 on the fp16 arithmetic: z sum_k a_k comes off the
+    // FP32 sums) is then a half-warp reduction in a fixed order, kept times 2^-24 (the subnormal
+    // codes' scale).
     constexpr bool kSub = kPost && std::is_same<MathT, __half>::value;
     const int Me = (M + 1) & ~1;
-    if constexpr (kSub) {
-        if (!wide) {
-            for (int item = warp; item < M * nneed; item += kGsAllWarps) {
-                const int m = item / nneed, sp = (sp0 + item - m * nneed) % steps;
-                const uint8_t* blk = acts + (uint32_t)m * RS + (uint32_t)sp * 320u + (uint32_t)(lane >> 3) * 80u +
-                                     (uint32_t)(lane & 7) * 8u;
-                const uint2 hv = *reinterpret_cast<const uint2*>(blk);
-                const __half2 h0 = *reinterpret_cast<const __half2*>(&hv.x), h1 = *reinterpret_cast<const __half2*>(&hv.y);
-                float v = (__low2float(h0) + __high2float(h0)) + (__low2float(h1) + __high2float(h1));
+    const int rot = (cta * 64) % nchunk;
+    auto chunk_of = [&](int c0, int& sp) {
+        int q = c0 + rot;
+        if (q >= nchunk) q -= nchunk;
+        sp = sp0 + (q >> 4);
+        if (sp >= steps) sp -= steps;
+        return 16 * sp + (q & 15);
+    };
+    auto chunk_off = [&](int m, int c) {
+        return (uint32_t)m * RS + (uint32_t)(c >> 4) * 320u + (uint32_t)((c >> 2) & 3) * 80u + (uint32_t)(c & 3) * 16u;
+    };
+    // sum of the unit over the half warp (a pass's bound on c0 is the same for all 16 lanes of a
+    // half, not always for the other half: hence the half's own mask); lane 0 of the half writes it
+    const uint32_t half_mask = 0xFFFFu << (lane & 16);
+    auto unit_sum = [&](float v, int m, int sp) {
+        v += __shfl_xor_sync(half_mask, v, 8);
+        v += __shfl_xor_sync(half_mask, v, 4);
+        v += __shfl_xor_sync(half_mask, v, 2);
+        v += __shfl_xor_sync(half_mask, v, 1);
+        if ((lane & 15) == 0) sa[sp * Me + m] = v * 5.9604644775390625e-08f;   // 2^-24
+    };
+    auto half8_sum = [](const uint4& v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float s8 = 0.0f;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) sa[sp * Me + m] = v * 5.9604644775390625e-08f;   // 2^-24
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+            s8 += __low2float(h) + __high2float(h);
+        }
+        return s8;
+    };
+    for (int m = 0; m < M; ++m) {
+        uint32_t emax = 0, emin = 255;   // largest, smallest nonzero biased exponent of row m
+        for (int c0 = threadIdx.x; c0 < nchunk; c0 += 4 * kGsThreads) {
+            uint4 vv[4];
+            int cc[4], sps[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (c0 + j * kGsThreads < nchunk) {
+                    cc[j] = chunk_of(c0 + j * kGsThreads, sps[j]);
+                    vv[j] = *reinterpret_cast<const uint4*>(A + (size_t)m * p.lda + 8 * cc[j]);
+                }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (c0 + j * kGsThreads < nchunk) {
+                    *reinterpret_cast<uint4*>(acts + chunk_off(m, cc[j])) = make_uint4(vv[j].x, vv[j].z, vv[j].y, vv[j].w);
+                    if constexpr (kConv) {
+                        const uint32_t x[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t e0 = (x[q] >> 7) & 0xFFu, e1 = (x[q] >> 23) & 0xFFu;
+                            emax = max(emax, max(e0, e1));
+                            if (x[q] & 0x7FFFu) emin = min(emin, e0);
+                            if (x[q] & 0x7FFF0000u) emin = min(emin, e1);
+                        }
+                    } else if constexpr (kSub) {
+                        unit_sum(half8_sum(vv[j]), m, sps[j]);
+                    }
+                }
+        }
+        if constexpr (kConv) {
+            emax = __reduce_max_sync(0xffffffffu, emax);
+            emin = __reduce_min_sync(0xffffffffu, emin);
+            if (lane == 0) {
+                atomicMax(&rowexp[m], (int)emax);
+                atomicMin(&rowmin[m], (int)emin);
             }
-            if (M & 1)
-                for (int q = threadIdx.x; q < nneed; q += kGsThreads) sa[((sp0 + q) % steps) * Me + M] = 0.0f;
-            __syncthreads();
         }
     }
+    if constexpr (kConv) {
+        // second pass, in shared memory: bf16 -> 2^-k * a in fp16, unless some row is too wide, and
+        // the unit sums of the converted values
+        __syncthreads();
+        for (int m = 0; m < M; ++m) wide = wide || rowexp[m] - rowmin[m] > 31;
+        for (int m = 0; m < M && !wide; ++m) {
+            const int k = min(max(rowexp[m] - 141, -100), 114);
+            const float down = __int_as_float((127 - k) << 23);
+            for (int c0 = threadIdx.x; c0 < nchunk; c0 += kGsThreads) {
+                int sp;
+                const int c = chunk_of(c0, sp);
+                uint4* q = reinterpret_cast<uint4*>(acts + chunk_off(m, c));
+                uint4 v = *q;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16) * down,
+                                                  __uint_as_float(w[i] & 0xFFFF0000u) * down);
+                    w[i] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                *q = v;
+                unit_sum(half8_sum(v), m, sp);
+            }
+        }
+    }
+    if constexpr (kSub)
+        if (M & 1)
+            for (int q = threadIdx.x; q < nneed; q += kGsThreads) {
+                int sp = sp0 + q;
+                if (sp >= steps) sp -= steps;
+                sa[sp * Me + M] = 0.0f;
+            }
+    __syncthreads();
 
     // activation fragments: lane holds row 8 b + g (rows at or past M read a zero block)
     const uint8_t* abase[NB];
