@@ -26,14 +26,23 @@
 // (g = lane / 4, t = lane % 4) reads the 16 bytes of block t (32 K) of channels 32 w + g + 8 r,
 // r = 0..3 (block t keeps channel n at slot n ^ 2t: the four lanes t of a channel hit different
 // banks), and the unit's activations of batch rows 8 b + g.
-//   Nibble pairs become 16-bit operands by one mask-OR with a magic exponent (fp16 0x6400 | u =
-//   1024 + u, 0x6400 | (u << 4) = 1024 + 16 u; bf16 0x4300 | u = 128 + u) and the zero point is
-//   subtracted exactly in 16 bits: group 128 scales the unit's FP32 sum once; groups 64 and 32
-//   (a lane's 32 K may span several groups) scale each operand first, (u - z) * s rounded once to
-//   the 16-bit type (bf16: s = s_hi + s_lo, both exact in bf16), and the MMAs accumulate the
-//   whole tile segment. (Codes fed to the MMA as fp16 subnormals u 2^-24, one AND per operand
-//   and the zero point taken off the FP32 sums with extra MMA chains on constant rows, cut the
-//   integer work but added half again as many MMAs, and measured 2% slower.)
+//   Group 128, fp16 arithmetic: one AND per operand leaves a code pair in the low mantissa bits of
+//   two fp16 subnormals, u 2^-24 (or 16 u 2^-24 for the upper nibble, kept in a second chain and
+//   scaled by 1/16 in FP32), which the MMA multiplies exactly; the zero point comes off the unit's
+//   FP32 sum as z * sum_k a_k (per-unit activation sums, formed while the activations are
+//   staged), and the scale multiplies it once. bf16 activations take this path too: each CTA
+//   scales every row by a power of two 2^-k (from the largest exponent among the row's staged
+//   values) and converts it to fp16 exactly, then multiplies its own sums by 2^k; when some row's
+//   values span more binades than fp16 holds, the CTA keeps bf16 and the next form.
+//   Other cases: one mask-OR with a magic exponent (fp16 0x6400 | u = 1024 + u, 0x6400 | (u << 4)
+//   = 1024 + 16 u; bf16 0x4300 | u = 128 + u) and an exact 16-bit subtraction of the zero point;
+//   group 128 scales the unit's FP32 sum once; groups 64 and 32 (a lane's 32 K may span several
+//   groups) scale each operand first, (u - z) * s rounded once to the 16-bit type (bf16: s = s_hi
+//   + s_lo, both exact in bf16), and the MMAs accumulate the whole tile segment.
+// Staging. Only the units of K that the CTA's range touches are staged. The producer issues the
+// first GS_PREFETCH stages before the activations are read and the rest of the ring after: a full
+// ring of weight copies issued by every SM at once is several microseconds of HBM traffic, and
+// the activation loads would queue behind it.
 // Every wait is bounded (the limit of w4a16_set_wait_limit_ns, 2 s by default); on expiry the
 // kernel records W4A16_ETIMEOUT, stops issuing copies, still passes every barrier and tile
 // counter, and lets the copies in flight land before it exits.
@@ -44,6 +53,10 @@
 #include "dequant.cuh"
 #include "sm100_ptx.cuh"
 #include "tiled_layout.cuh"
+
+#ifndef GS_PREFETCH
+#define GS_PREFETCH 2
+#endif
 
 namespace w4a16 {
 namespace {
@@ -184,8 +197,9 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         ++issued[s];
     };
     const bool producer = warp == kGsWarpProducer && lane == 0;
+    const int npre = min(min(nst, ns), GS_PREFETCH);
     if (producer)
-        for (int st = 0; st < nst && st < ns; ++st) issue(st);
+        for (int st = 0; st < npre; ++st) issue(st);
 
     const int grp = warp / kGsGroupWarps, wg = warp % kGsGroupWarps;
     const int g = lane >> 2, t = lane & 3;
@@ -509,6 +523,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         // ------------------------------------------------------------ producer (lane 0)
         // refills slot s with stage st once the 16 compute warps have left stage st - ns
         if (lane == 0) {
+            for (int st = npre; st < nst && st < ns; ++st) issue(st);
             for (int st = ns; st < nst; ++st) {
                 if (!mbar_wait(&empty[st % ns], (uint32_t)((st / ns) - 1) & 1u, abort_flag, p.dev_status, p.wait_ns))
                     break;
