@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) fp8_wquant_kernel(const uint16_t* __restr
         const int k = k0 + r, n = n0 + tx;
         t[r][tx] = e4m3_rn(f16_bits_to_f64(W[(size_t)k * N + n]) / (double)sw[n]);
     }
-    __syncthreads();
+    cta_sync();
     for (int r = ty; r < 32; r += 8) Wq[(size_t)(n0 + r) * K + k0 + tx] = t[tx][r];
 }
 
@@ -91,10 +91,10 @@ __global__ void __launch_bounds__(256) fp8_aquant_kernel(const uint16_t* __restr
     double amax = 0.0;
     for (int k = threadIdx.x; k < K; k += 256) amax = fmax(amax, fabs(act_to_f64<T>(row[k])));
     red[threadIdx.x] = amax;
-    __syncthreads();
+    cta_sync();
     for (int w = 128; w > 0; w >>= 1) {
         if (threadIdx.x < w) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + w]);
-        __syncthreads();
+        cta_sync();
     }
     const float s = scale_from_amax(red[0]);
     if (threadIdx.x == 0) sa[m] = s;
@@ -147,7 +147,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    cta_sync();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
 
@@ -205,7 +205,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     }
 
     tc_fence_before();
-    __syncthreads();
+    cta_sync();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_d, Cfg::kTmemCols);

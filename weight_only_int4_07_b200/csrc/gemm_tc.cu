@@ -168,7 +168,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    cta_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tmem_w = tmem + (uint32_t)(2 * kCols);   // the step ring's weight tiles
@@ -433,7 +433,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     }
 
     tc_fence_before();
-    __syncthreads();
+    cta_sync();
     if (warp == kTcWarpLoadA) {
         tc_fence_after();
         tmem_dealloc(tmem, kTcTmemCols);

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     for (int i = threadIdx.x; i < 96; i += kGsThreads) reinterpret_cast<uint32_t*>(zrow)[i] = 0u;
     if (threadIdx.x < 2) reinterpret_cast<uint32_t*>(zrow + 448)[threadIdx.x] = 0u;   // two zero sums
     if (threadIdx.x < 16) rowmin[threadIdx.x] = 255;
-    __syncthreads();
+    cta_sync();
     grid_dependents_launch();
 
     // stage st = records u0 + 4 st .. (up to 4), one bulk copy into slot st % ns
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     if constexpr (kConv) {
         // second pass, in shared memory: bf16 -> 2^-k * a in fp16, unless some row is too wide, and
         // the unit sums of the converted values
-        __syncthreads();
+        cta_sync();
         for (int m = 0; m < M; ++m) wide = wide || rowexp[m] - rowmin[m] > 31;
         for (int m = 0; m < M && !wide; ++m) {
             const int k = min(max(rowexp[m] - 141, -100), 114);
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                 if (sp >= steps) sp -= steps;
                 sa[sp * Me + M] = 0.0f;
             }
-    __syncthreads();
+    cta_sync();
 
     // activation fragments: lane holds row 8 b + g (rows at or past M read a zero block)
     const uint8_t* abase[NB];
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
 
     // after a timeout: let every copy still in flight land before the CTA exits (a wait that does
     // not give up on the raised abort flag, still bounded in time); only the producer issues copies
-    __syncthreads();
+    cta_sync();
     if (producer && *abort_flag) {
         volatile int keep_waiting = 0;
         for (int s = 0; s < ns; ++s)

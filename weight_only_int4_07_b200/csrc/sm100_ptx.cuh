@@ -22,6 +22,14 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// CTA-wide barrier that each thread passes on its own (the non-.aligned form): correct after
+// role code in which one lane of a warp runs on (a producer's issue loop, an elected MMA issuer)
+// while its other lanes have already reached the barrier. __syncthreads is the .aligned form,
+// whose behaviour is undefined unless every lane of a warp executes it together.
+__device__ __forceinline__ void cta_sync() {
+    asm volatile("barrier.sync 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
