@@ -10,9 +10,10 @@
 // of bytes. One CTA per SM takes floor(U / P) or ceil(U / P) consecutive units. A tile whose units
 // all belong to one CTA is written straight to C. A tile cut between CTAs cf < ... < cl is the
 // last tile of cf's range and the first of every later one: each later CTA publishes its FP32
-// sums to the workspace and counts them (release, no wait) as soon as it has them; cf, at the end
-// of its range, waits for the count (acquire, bounded), adds the sums in CTA order, writes C and
-// resets the counter. The result does not depend on timing.
+// sums to the workspace and counts them (release, no wait) as soon as it has them; cf's epilogue
+// warp, while cf's compute warps are still on the tile, waits for the count (acquire, bounded),
+// adds the later CTAs' sums in CTA order and resets the counter; cf's own sums plus that total
+// go to C. The result does not depend on timing.
 //
 // Pipeline. Stages of up to 4 records (34 KiB at group 128) are filled by one bulk copy each.
 // Sixteen compute warps in four groups: group q takes unit q of every stage, warp w of a group
@@ -541,46 +542,37 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                                                                             : nunits;
         for (int et = 0; elo < nunits; ++et) {
             const int bsel = et & 1;
-            (void)wait_uniform(&tfull[bsel], (uint32_t)(et >> 1) & 1u, abort_flag, p.dev_status, p.wait_ns);
-            const float* rb = red + (size_t)bsel * kGsGroups * M * 128;
             const size_t n0 = (size_t)etile * 128;
             const int cf = unit_owner((long long)etile * steps, U, P);
             const int cl = unit_owner((long long)etile * steps + steps - 1, U, P);
-            if (cf == cl || cta == cf) {
-                if (cf != cl) {
-                    // the tile is cut between CTAs cf .. cl and this is cf: the tile is the last of
-                    // its range. Wait until every later CTA of the tile has published its sums (they
-                    // hold the tile at the start of their ranges), then add them in CTA order.
-                    if (lane == 0) {
-                        const uint64_t t0 = globaltimer_ns();
-                        for (;;) {
-                            int n;
-                            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + etile)
-                                         : "memory");
-                            if (n >= cl - cf) break;
-                            if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
-                                *abort_flag = 1;
-                                report_status(p.dev_status, W4A16_ETIMEOUT);
-                                break;
-                            }
+            // The tile is cut between CTAs cf .. cl and this is cf: the tile is the last of this
+            // range, and the later CTAs hold it at the start of theirs. Before this CTA's own sums
+            // are in, wait until they have all published theirs and add them up, in CTA order, into
+            // the other shared buffer (free: no tile follows), so that reaching them from L2 is off
+            // the path once the compute warps finish.
+            const bool gather = cf != cl && cta == cf;
+            float* pre = red + (size_t)(bsel ^ 1) * kGsGroups * M * 128;
+            if (gather) {
+                if (lane == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    for (;;) {
+                        int n;
+                        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + etile)
+                                     : "memory");
+                        if (n >= cl - cf) break;
+                        if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+                            *abort_flag = 1;
+                            report_status(p.dev_status, W4A16_ETIMEOUT);
+                            break;
                         }
-                        p.counters[etile] = 0;
                     }
-                    __syncwarp();
+                    p.counters[etile] = 0;
                 }
+                __syncwarp();
                 for (int m = 0; m < M; ++m) {
-                    float up = 1.0f;
-                    if constexpr (kConv)   // undo the row's 2^-k
-                        if (!wide) up = __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
-                    float y[4];   // this CTA's sums, back in the scale of A
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int ch = lane + 32 * j;
-                        y[j] = (rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
-                                rb[(3 * M + m) * 128 + ch]) * up;
-                    }
-                    // the later CTAs' sums, in CTA order; the loads of four CTAs in flight together
-                    for (int c0 = cf + 1; cf != cl && c0 <= cl; c0 += 4) {
+                    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    // the loads of four CTAs in flight together
+                    for (int c0 = cf + 1; c0 <= cl; c0 += 4) {
                         float ld[4][4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -595,9 +587,24 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                                 if (c0 + q <= cl) y[j] += ld[q][j];
                     }
 #pragma unroll
+                    for (int j = 0; j < 4; ++j) pre[m * 128 + lane + 32 * j] = y[j];
+                }
+            }
+            (void)wait_uniform(&tfull[bsel], (uint32_t)(et >> 1) & 1u, abort_flag, p.dev_status, p.wait_ns);
+            const float* rb = red + (size_t)bsel * kGsGroups * M * 128;
+            if (cf == cl || cta == cf) {
+                for (int m = 0; m < M; ++m) {
+                    float up = 1.0f;
+                    if constexpr (kConv)   // undo the row's 2^-k
+                        if (!wide) up = __int_as_float((127 + min(max(rowexp[m] - 141, -100), 114)) << 23);
+#pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int ch = lane + 32 * j;
-                        const float o = y[j];
+                        // this CTA's sums, back in the scale of A, then the later CTAs' (a lane
+                        // reads back only what it wrote)
+                        float o = (rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
+                                   rb[(3 * M + m) * 128 + ch]) * up;
+                        if (gather) o += pre[m * 128 + ch];
                         if (p.out_f32)
                             p.out_f32[(size_t)m * N + n0 + ch] = o;
                         else
