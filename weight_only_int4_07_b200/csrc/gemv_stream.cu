@@ -679,9 +679,10 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                     }
                 }
             }
-            // leave the stage: this warp's reads of the slot were consumed by its MMAs
+            // leave the stage: this warp's reads of the slot were consumed by its MMAs (after
+            // giving up, no more: the slot may still have a copy in flight, not to be reissued)
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s_idx]);
+            if (lane == 0 && !aborted) mbar_arrive(&empty[s_idx]);
         }
         while (seg_lo < nunits) tile_end();
     }
