@@ -639,18 +639,20 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
         }
     } else {
         // ------------------------------------------------------------ compute warps
+        // Group grp takes unit 4 st + grp of stage st. The loop runs over the tile segments of the
+        // range, each ended by tile_end outside the unit loop (which keeps its registers to
+        // itself); the units of consecutive segments are consecutive stages. A group with no unit
+        // in the last stage neither waits for it nor leaves it: no copy refills the last stage.
         bool aborted = false;
         int s_idx = -1;
         uint32_t ph = 0;
-        for (int st = 0; st < nst; ++st) {
-            if (++s_idx == ns) {
-                s_idx = 0;
-                ph ^= 1u;
-            }
-            if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status, p.wait_ns)) aborted = true;
-            const int li = st * kGsUnitsPerStage + grp;
-            if (li < nunits) {
-                while (li >= seg_hi) tile_end();
+        for (;;) {
+            for (int li = seg_lo + ((grp - seg_lo) & 3); li < seg_hi; li += kGsUnitsPerStage) {
+                if (++s_idx == ns) {
+                    s_idx = 0;
+                    ph ^= 1u;
+                }
+                if (!aborted && !wait_uniform(&full[s_idx], ph, abort_flag, p.dev_status, p.wait_ns)) aborted = true;
                 if (!aborted) {
                     const int sp = sp_lo + (li - seg_lo);
                     const uint8_t* rec = stages + (uint32_t)s_idx * stage_bytes + rec_off;
@@ -678,13 +680,14 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                         unit_math(OpsTag<Ops>{}, km, cw, sb, zw, v);
                     }
                 }
+                // leave the stage: this warp's reads of the slot were consumed by its MMAs (after
+                // giving up, no more: the slot may still have a copy in flight, not to be reissued)
+                __syncwarp();
+                if (lane == 0 && !aborted) mbar_arrive(&empty[s_idx]);
             }
-            // leave the stage: this warp's reads of the slot were consumed by its MMAs (after
-            // giving up, no more: the slot may still have a copy in flight, not to be reissued)
-            __syncwarp();
-            if (lane == 0 && !aborted) mbar_arrive(&empty[s_idx]);
+            tile_end();
+            if (seg_lo >= nunits) break;
         }
-        while (seg_lo < nunits) tile_end();
     }
 
     // after a timeout: let every copy still in flight land before the CTA exits (a wait that does
