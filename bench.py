@@ -48,7 +48,7 @@ METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=256, as % of B200 roofline"
 SWEEP_MS = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 2048)
 # ncu DRAM traffic of the decode kernel, written by hand from a capture into this file, with the
 # hash of the kernel sources it was taken on (the bench reports it only while they match)
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_stream_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_stream_traffic.txt")   # JSON
 DECODE_SOURCES = ("gemv_stream.cu", "sm100_ptx.cuh", "tiled_layout.cuh", "common.cuh")
 
 
