@@ -179,16 +179,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             int rs = 0, issued[kTcMaxRing];
             uint32_t rph = 0;
             for (int i = 0; i < nr; ++i) issued[i] = 0;
+            // unit i = tile tau (channel tile nt, row block mb), step ku (kept by increments)
+            const long long tau0 = u0 / UT;
+            int ku = (int)(u0 - tau0 * UT), mb = (int)(tau0 % p.mblocks);
+            long long nt = tau0 / p.mblocks;
             for (long long i = u0; i < u1;) {
-                const long long tau = i / UT;
-                const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
-                const int n = (int)(seg_end - i < kTcUnitsPerLoad ? seg_end - i : kTcUnitsPerLoad);
+                const int n = UT - ku < kTcUnitsPerLoad ? (u1 - i < UT - ku ? (int)(u1 - i) : UT - ku)
+                                                         : (u1 - i < kTcUnitsPerLoad ? (int)(u1 - i) : kTcUnitsPerLoad);
                 if (!mbar_wait(&empty_r[rs], rph ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
-                const long long rec = (tau / p.mblocks) * UT + (i - tau * UT);
+                const long long rec = nt * UT + ku;
                 mbar_arrive_expect_tx(&full_r[rs], (uint32_t)n * R);
                 bulk_g2s(ring_w + (size_t)rs * p.slot_w, p.tiled + (size_t)rec * R, (uint32_t)n * R, &full_r[rs]);
                 ++issued[rs];
                 i += n;
+                if ((ku += n) == UT) {
+                    ku = 0;
+                    if (++mb == p.mblocks) {
+                        mb = 0;
+                        ++nt;
+                    }
+                }
                 if (++rs == nr) {
                     rs = 0;
                     rph ^= 1u;
@@ -207,10 +217,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             for (int i = 0; i < NS; ++i) issued[i] = 0;
             int s = 0;
             uint32_t ph = 0;
+            // unit i = tile tau, step ku; row block mb = tau mod mblocks (kept by increments)
+            long long tau0 = u0 / UT;
+            int ku = (int)(u0 - tau0 * UT), mb = (int)(tau0 % p.mblocks);
             for (long long i = u0; i < u1; ++i) {
-                const long long tau = i / UT;
-                const int mb = (int)(tau % p.mblocks);
-                const int ku = (int)(i - tau * UT);
+                if (i > u0 && ++ku == UT) {
+                    ku = 0;
+                    if (++mb == p.mblocks) mb = 0;
+                }
                 if (!mbar_wait(&free_s[s], ph ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
                 mbar_arrive_expect_tx(&full_a[s], kSlotA);
                 uint8_t* dst = ring_a + (size_t)s * kSlotA;
@@ -380,11 +394,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         int rs = 0, s = 0;
         uint32_t rph = 0, ph = 0;
         bool ok = true;
+        long long tend = (u0 / UT + 1) * UT;   // end of the current tile's units
         for (long long i = u0; i < u1 && ok;) {
-            const long long tau = i / UT;
-            const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
+            const long long seg_end = u1 < tend ? u1 : tend;
             const int nu = (int)(seg_end - i < kTcUnitsPerLoad ? seg_end - i : kTcUnitsPerLoad);
             i += nu;
+            if (i == tend) tend += UT;
             if (!tc_wait(&full_r[rs], rph, abort_flag, p.dev_status, wait_ns)) {
                 ok = false;
                 break;
