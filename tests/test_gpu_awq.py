@@ -1,7 +1,7 @@
 """AWQ on the GPU (w4a16_awq_quantize) against the FP64 oracle ("4.3 Weight-only INT4",
-section 3): codes, scales, zeros and input factors bit for bit on full small layers; at a larger
-size, a lower layer-output error than RTN and the encoded layer running through the fused GEMM
-(inputs divided by the factors) within the bound."""
+section 3): codes, scales, zeros and input factors bit for bit on full small layers and on a
+2048 x 2048 layer; at that size also a lower layer-output error than RTN and the encoded layer
+running through the fused GEMM (inputs divided by the factors) within the bound."""
 import numpy as np
 import pytest
 import torch
@@ -43,6 +43,24 @@ def _np(t, dt):
 def test_awq_bit_exact_full(K, N, S, group, sym, x_dtype):
     Wb = synthetic.weights_normal(K, N, 400 + K)
     Xb = synthetic.calibration(S, K, 401 + K, dtype=x_dtype, outlier_frac=0.02, outlier_mult=20.0)
+    oc, os_, oz, osb, ai = oawq.awq(Wb, Xb, x_dtype, group, sym)
+    gc, gs, gz, gsi = native.w4a16_awq_quantize(_dev16(Wb, synthetic.F16), _dev16(Xb, x_dtype), group, sym)
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(gsi.view(torch.int16), np.uint16), osb)
+    assert np.array_equal(_np(gs.view(torch.int16), np.uint16), os_)
+    assert np.array_equal(_np(gc, np.int32), oc)
+    if not sym:
+        assert np.array_equal(_np(gz, np.int32), oz)
+
+
+@pytest.mark.parametrize("sym,x_dtype", [(0, 0), (1, 1)])
+def test_awq_bit_exact_2048(sym, x_dtype):
+    """A 2048 x 2048 layer with 512 calibration rows (the size of the error test below): the
+    factors, codes, scales and zeros bit for bit against the oracle, whose alpha and clip
+    searches take every candidate over the whole layer."""
+    K, N, S, group = 2048, 2048, 512, 128
+    Wb = synthetic.weights_normal(K, N, 420 + sym)
+    Xb = synthetic.calibration(S, K, 421 + sym, dtype=x_dtype, outlier_frac=0.02, outlier_mult=20.0)
     oc, os_, oz, osb, ai = oawq.awq(Wb, Xb, x_dtype, group, sym)
     gc, gs, gz, gsi = native.w4a16_awq_quantize(_dev16(Wb, synthetic.F16), _dev16(Xb, x_dtype), group, sym)
     torch.cuda.synchronize()
