@@ -28,10 +28,13 @@
 //   warp 1      : activation loader -- per 128-K step (one unit), two TMA boxes of BN rows x
 //                 64 K into the step's slot of a ring (4-7 slots: the tiles come from L2, and a
 //                 slot stays busy until its MMAs complete); owns the tensor memory.
-//   warp 2      : MMA issuer -- one thread issues the eight tcgen05.mma (K = 16 each) of a step,
-//                 operand A (the weights) from tensor memory and B (the activations) from shared
-//                 memory, and one commit that frees the step's activation and weight tiles
-//                 together; after a tile's last step a commit to the accumulator.
+//   warps 2, 3  : MMA issuers (two below BN = 128, one at 128) -- lane 0 of warp 2 + j takes the
+//                 units j, j + 2, .. of the range:
+//                 the eight tcgen05.mma (K = 16 each) of a step, operand A (the weights) from
+//                 tensor memory and B (the activations) from shared memory, into issuer j's own
+//                 accumulator of the tile, and one commit that frees the step's activation and
+//                 weight tiles together; after a tile's last step a commit to the tile's barrier
+//                 (one arrival per issuer). The epilogue adds the accumulators.
 //   warps 4..7  : epilogue -- tcgen05.ld of the accumulator (warp w reads lanes 32 (w % 4) ..),
 //                 then C (or the published partial sums of a cut tile); two accumulators, so one
 //                 tile's epilogue runs under the next tile's MMAs.
@@ -40,8 +43,8 @@
 //                 tcgen05.st into a ring of weight tiles in tensor memory (lane n = channel n, 64
 //                 columns of K pairs per 128-K step); warp w writes the lanes 32 (w % 4) .. its
 //                 channels occupy.
-// Tensor memory (512 columns): two accumulators (BN <= 128 columns each), then the weight tiles
-// of the step ring (64 columns per step). A has at most 128 rows per tile; more rows of A are
+// Tensor memory (512 columns): two tiles in flight, each with one accumulator per issuer (BN <=
+// 128 columns), then the weight tiles of the step ring (64 columns per step). A has at most 128 rows per tile; more rows of A are
 // more tiles (row blocks), whose weights are dequantized again but read from L2.
 // Record slots are freed by the dequant warps, activation and weight-tile slots by the MMA
 // commits, so the weight stream runs several units ahead of the tensor cores, and the shared
@@ -74,11 +77,17 @@ constexpr int kTcMaxRing = 16;
 constexpr int kTcTmemCols = 512;
 constexpr int kTcStepCols = 64;        // tensor-memory columns of one 128-K weight tile (K pairs)
 
-// Two accumulators (BN columns each, at least 32) in tensor memory, then the step ring's weight
-// tiles: as many as fit, at most 8.
+// MMA threads: two below BN = 128 (issuer j takes the units j, j + 2, .. of the range; at small N
+// one thread's issue rate, not the tensor pipe, sets the time), one at BN = 128. Tensor memory:
+// two tiles in flight (one tile's epilogue runs under the next tile's MMAs), each with one
+// accumulator per issuer (BN columns, at least 32), then the step ring's weight tiles: as many
+// as fit, at most 8.
+__host__ __device__ constexpr int tc_issuers(int bn) { return bn >= 128 ? 1 : 2; }
 __host__ __device__ constexpr int tc_acc_cols(int bn) { return bn < 32 ? 32 : bn; }
 __host__ __device__ constexpr int tc_steps(int bn) {
-    return (kTcTmemCols - 2 * tc_acc_cols(bn)) / kTcStepCols > 8 ? 8 : (kTcTmemCols - 2 * tc_acc_cols(bn)) / kTcStepCols;
+    return (kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols > 8
+               ? 8
+               : (kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols;
 }
 constexpr uint64_t kTcDrainNs = 2000000000ull;
 
@@ -117,6 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     using Ops = GsOps<T>;
     constexpr int kCols = tc_acc_cols(BN);       // tensor-memory columns of one accumulator
+    constexpr int kIss = tc_issuers(BN);         // MMA threads
     constexpr int NS = tc_steps(BN);             // steps in flight (activation + weight tiles)
     constexpr uint32_t kSlotA = (uint32_t)BN * 256u;   // 128 K of BN rows: two 64-K TMA boxes
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -156,10 +166,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             mbar_init(&free_s[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&accfull[i], 1);
+            mbar_init(&accfull[i], kIss);
             mbar_init(&accempty[i], 4);
         }
-        mbar_init(lastmma, 1);
+        mbar_init(lastmma, kIss);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -171,7 +181,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     cta_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_w = tmem + (uint32_t)(2 * kCols);   // the step ring's weight tiles
+    const uint32_t tmem_w = tmem + (uint32_t)(2 * kIss * kCols);   // the step ring's weight tiles
 
     if (warp == kTcWarpLoadW) {
         // ------------------------------------------------------------ weight records
@@ -240,9 +250,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             for (int q = 0; q < NS; ++q)
                 if (issued[q] > 0) mbar_wait(&full_a[q], (uint32_t)(issued[q] - 1) & 1u, &keep, nullptr, kTcDrainNs);
         }
-    } else if (warp == kTcWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp >= kTcWarpMma && warp < kTcWarpMma + kIss) {
+        // ------------------------------------------------------------ MMA issuers
+        // Issuer j (lane 0 of warp kTcWarpMma + j) takes the units j, j + kIss, .. of the range into
+        // its own accumulator of the tile; the epilogue adds them. (One thread issuing all the
+        // MMAs measured about 1.1k cycles per unit at N = 16, the tensor pipe mostly idle.)
         if (lane == 0) {
+            const int j = warp - kTcWarpMma;
             constexpr uint32_t idesc = idesc_f16(BN, std::is_same<T, __nv_bfloat16>::value);
             int s = 0, use[2] = {0, 0}, ab = 0;
             uint32_t ph = 0;
@@ -252,34 +266,37 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
                 if (!mbar_wait(&accempty[ab], ((uint32_t)use[ab] & 1u) ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(ab * kCols);
+                const uint32_t d_tmem = tmem + (uint32_t)((ab * kIss + j) * kCols);
                 bool first = true;
                 for (; i < seg_end; ++i) {
-                    if (!mbar_wait(&full_d[s], ph, abort_flag, p.dev_status, wait_ns) ||
-                        !mbar_wait(&full_a[s], ph, abort_flag, p.dev_status, wait_ns)) {
-                        ok = false;
-                        break;
+                    if (kIss == 1 || (int)((i - u0) & 1) == j) {
+                        if (!mbar_wait(&full_d[s], ph, abort_flag, p.dev_status, wait_ns) ||
+                            !mbar_wait(&full_a[s], ph, abort_flag, p.dev_status, wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // the unit's eight K-steps of 16: weights from tensor memory, activations
+                        // from the two 64-K boxes of the step's tile; one commit frees both tiles
+                        const uint32_t a_tm = tmem_w + (uint32_t)(s * kTcStepCols);
+                        const uint32_t b_sm = smem_u32(ring_a + (size_t)s * kSlotA);
+                        mma4_f16_ts(d_tmem, a_tm, smem_desc_sw128(b_sm), idesc, first ? 0u : 1u);
+                        mma4_f16_ts(d_tmem, a_tm + 32u, smem_desc_sw128(b_sm + kSlotA / 2), idesc, 1u);
+                        mma_commit(&free_s[s]);
+                        first = false;
                     }
-                    tc_fence_after();
-                    // the unit's eight K-steps of 16: weights from tensor memory, activations from
-                    // the two 64-K boxes of the step's tile; one commit frees both tiles
-                    const uint32_t a_tm = tmem_w + (uint32_t)(s * kTcStepCols);
-                    const uint32_t b_sm = smem_u32(ring_a + (size_t)s * kSlotA);
-                    mma4_f16_ts(d_tmem, a_tm, smem_desc_sw128(b_sm), idesc, first ? 0u : 1u);
-                    mma4_f16_ts(d_tmem, a_tm + 32u, smem_desc_sw128(b_sm + kSlotA / 2), idesc, 1u);
-                    mma_commit(&free_s[s]);
-                    first = false;
                     if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
+                // (with no unit of this tile, the commit arrives at once)
                 mma_commit(&accfull[ab]);
                 ++use[ab];
                 ab ^= 1;
             }
-            // the CTA exits only after its last MMAs completed
+            // the CTA exits only after the last MMAs of every issuer completed
             mma_commit(lastmma);
             volatile int keep = 0;
             mbar_wait(lastmma, 0, &keep, nullptr, kTcDrainNs);
@@ -295,14 +312,36 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         for (long long i = u0; i < u1;) {
             const long long tau = i / UT;
             const long long seg_end = u1 < (tau + 1) * UT ? u1 : (tau + 1) * UT;
-            i = seg_end;
+            // the issuers that hold units of this tile segment (issuer j: units j, j + 2, ..)
+            const long long seg_lo = i;
+            const bool has0 = kIss == 1 || seg_end - seg_lo >= 2 || ((seg_lo - u0) & 1) == 0;
+            const bool has1 = kIss == 2 && (seg_end - seg_lo >= 2 || ((seg_lo - u0) & 1) == 1);
             ok = ok && tc_wait(&accfull[ab], (uint32_t)use[ab] & 1u, abort_flag, p.dev_status, wait_ns);
             tc_fence_after();
             const int nt = (int)(tau / p.mblocks), mb = (int)(tau % p.mblocks);
             const size_t n0 = (size_t)nt * 128;
             const int m0 = mb * BN;
             const int cf = tc_unit_owner(tau * UT, U, P), cl = tc_unit_owner(tau * UT + UT - 1, U, P);
-            const uint32_t lane_base = tmem + (uint32_t)(ab * kCols) + ((uint32_t)(32 * q) << 16);
+            i = seg_end;
+            const uint32_t lane_base = tmem + (uint32_t)(ab * kIss * kCols) + ((uint32_t)(32 * q) << 16);
+            // the tile's FP32 sums, 16 columns from c: the issuers' accumulators added
+            auto acc16 = [&](int c, float (&y)[16]) {
+                uint32_t v[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) y[jj] = 0.0f;
+                if (has0) {
+                    tmem_ld16(lane_base + (uint32_t)(c * 16), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) y[jj] = __uint_as_float(v[jj]);
+                }
+                if (has1) {
+                    tmem_ld16(lane_base + (uint32_t)(kCols + c * 16), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) y[jj] += __uint_as_float(v[jj]);
+                }
+            };
             if (cf == cl || cta == cf) {
                 if (cf != cl) {
                     // the tile is cut between CTAs cf .. cl and this is cf: wait until every later
@@ -327,12 +366,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 if (ok && !*abort_flag) {
 #pragma unroll 1
                     for (int c = 0; c < BN / 16; ++c) {
-                        uint32_t v[16];
-                        tmem_ld16(lane_base + (uint32_t)(c * 16), v);
-                        tmem_ld_wait();
                         float y[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(v[j]);
+                        acc16(c, y);
                         // the other CTAs' sums, in CTA order; the 16 loads of one CTA in flight together
 #pragma unroll 1
                         for (int cc = cf + 1; cc <= cl; ++cc) {
@@ -357,13 +392,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                     float* part = p.partials + (size_t)cta * BN * 128;
 #pragma unroll 1
                     for (int c = 0; c < BN / 16; ++c) {
-                        uint32_t v[16];
-                        tmem_ld16(lane_base + (uint32_t)(c * 16), v);
-                        tmem_ld_wait();
+                        float y[16];
+                        acc16(c, y);
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int mr = c * 16 + j;
-                            if (m0 + mr < p.M) __stcg(part + (size_t)mr * 128 + n, __uint_as_float(v[j]));
+                            if (m0 + mr < p.M) __stcg(part + (size_t)mr * 128 + n, y[j]);
                         }
                     }
                 }
