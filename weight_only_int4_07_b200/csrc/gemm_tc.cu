@@ -43,9 +43,10 @@
 //                 tcgen05.st into a ring of weight tiles in tensor memory (lane n = channel n, 64
 //                 columns of K pairs per 128-K step); warp w writes the lanes 32 (w % 4) .. its
 //                 channels occupy.
-// Tensor memory (512 columns): two tiles in flight, each with one accumulator per issuer (BN <=
-// 128 columns), then the weight tiles of the step ring (64 columns per step). A has at most 128 rows per tile; more rows of A are
-// more tiles (row blocks), whose weights are dequantized again but read from L2.
+// Tensor memory (512 columns): two tiles in flight (one at BN = 256), each with one accumulator per
+// issuer (BN columns), then the weight tiles of the step ring (64 columns per step). A has at
+// most 256 rows per tile (one MMA of N = 256 per K step); more rows of A are more tiles (row
+// blocks), whose weights are dequantized again but read from L2.
 // Record slots are freed by the dequant warps, activation and weight-tile slots by the MMA
 // commits, so the weight stream runs several units ahead of the tensor cores, and the shared
 // memory holds only copies in flight (weight records and activation tiles).
@@ -71,23 +72,28 @@ using namespace sm100;
 constexpr int kTcThreads = 768;
 constexpr int kTcWarpLoadW = 0, kTcWarpLoadA = 1, kTcWarpMma = 2, kTcWarpEpi = 4, kTcWarpDeq = 8;
 constexpr int kTcDeqWarps = 16;
-constexpr int kTcUnitsPerLoad = 2;     // unit records per record slot (one bulk copy)
+// unit records per record slot (one bulk copy): two, one at BN = 256 (whose activation tiles take
+// most of the shared memory)
+__host__ __device__ constexpr int tc_units_per_load(int bn) { return bn >= 256 ? 1 : 2; }
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcMaxRing = 16;
 constexpr int kTcTmemCols = 512;
 constexpr int kTcStepCols = 64;        // tensor-memory columns of one 128-K weight tile (K pairs)
 
 // MMA threads: two below BN = 128 (issuer j takes the units j, j + 2, .. of the range; at small N
-// one thread's issue rate, not the tensor pipe, sets the time), one at BN = 128. Tensor memory:
-// two tiles in flight (one tile's epilogue runs under the next tile's MMAs), each with one
-// accumulator per issuer (BN columns, at least 32), then the step ring's weight tiles: as many
-// as fit, at most 8.
+// one thread's issue rate, not the tensor pipe, sets the time), one from BN = 128. Tensor memory:
+// two tiles in flight below BN = 256 (one tile's epilogue runs under the next tile's MMAs), one
+// at 256, each with one accumulator per issuer (BN columns, at least 32), then the step ring's
+// weight tiles: as many as fit, at most 8; at BN = 256 three (the shared memory holds three
+// activation tiles of 64 KiB).
 __host__ __device__ constexpr int tc_issuers(int bn) { return bn >= 128 ? 1 : 2; }
+__host__ __device__ constexpr int tc_acc_bufs(int bn) { return bn >= 256 ? 1 : 2; }
 __host__ __device__ constexpr int tc_acc_cols(int bn) { return bn < 32 ? 32 : bn; }
 __host__ __device__ constexpr int tc_steps(int bn) {
-    return (kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols > 8
-               ? 8
-               : (kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols;
+    return bn >= 256 ? 3
+                     : ((kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols > 8
+                            ? 8
+                            : (kTcTmemCols - 2 * tc_issuers(bn) * tc_acc_cols(bn)) / kTcStepCols);
 }
 constexpr uint64_t kTcDrainNs = 2000000000ull;
 
@@ -127,6 +133,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     using Ops = GsOps<T>;
     constexpr int kCols = tc_acc_cols(BN);       // tensor-memory columns of one accumulator
     constexpr int kIss = tc_issuers(BN);         // MMA threads
+    constexpr int kBufs = tc_acc_bufs(BN);       // tiles in flight
+    constexpr int kUPL = tc_units_per_load(BN);  // unit records per record slot
     constexpr int NS = tc_steps(BN);             // steps in flight (activation + weight tiles)
     constexpr uint32_t kSlotA = (uint32_t)BN * 256u;   // 128 K of BN rows: two 64-K TMA boxes
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -181,7 +189,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
     cta_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_w = tmem + (uint32_t)(2 * kIss * kCols);   // the step ring's weight tiles
+    const uint32_t tmem_w = tmem + (uint32_t)(kBufs * kIss * kCols);   // the step ring's weight tiles
 
     if (warp == kTcWarpLoadW) {
         // ------------------------------------------------------------ weight records
@@ -194,8 +202,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             int ku = (int)(u0 - tau0 * UT), mb = (int)(tau0 % p.mblocks);
             long long nt = tau0 / p.mblocks;
             for (long long i = u0; i < u1;) {
-                const int n = UT - ku < kTcUnitsPerLoad ? (u1 - i < UT - ku ? (int)(u1 - i) : UT - ku)
-                                                         : (u1 - i < kTcUnitsPerLoad ? (int)(u1 - i) : kTcUnitsPerLoad);
+                const int n = UT - ku < kUPL ? (u1 - i < UT - ku ? (int)(u1 - i) : UT - ku)
+                                              : (u1 - i < kUPL ? (int)(u1 - i) : kUPL);
                 if (!mbar_wait(&empty_r[rs], rph ^ 1u, abort_flag, p.dev_status, wait_ns)) break;
                 const long long rec = nt * UT + ku;
                 mbar_arrive_expect_tx(&full_r[rs], (uint32_t)n * R);
@@ -294,7 +302,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
                 // (with no unit of this tile, the commit arrives at once)
                 mma_commit(&accfull[ab]);
                 ++use[ab];
-                ab ^= 1;
+                if (kBufs == 2) ab ^= 1;
             }
             // the CTA exits only after the last MMAs of every issuer completed
             mma_commit(lastmma);
@@ -409,7 +417,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[ab]);
             ++use[ab];
-            ab ^= 1;
+            if (kBufs == 2) ab ^= 1;
         }
     } else if (warp >= kTcWarpDeq) {
         // ------------------------------------------------------------ dequantize
@@ -431,7 +439,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const TcParams p) {
         long long tend = (u0 / UT + 1) * UT;   // end of the current tile's units
         for (long long i = u0; i < u1 && ok;) {
             const long long seg_end = u1 < tend ? u1 : tend;
-            const int nu = (int)(seg_end - i < kTcUnitsPerLoad ? seg_end - i : kTcUnitsPerLoad);
+            const int nu = (int)(seg_end - i < kUPL ? seg_end - i : kUPL);
             i += nu;
             if (i == tend) tend += UT;
             if (!tc_wait(&full_r[rs], rph, abort_flag, p.dev_status, wait_ns)) {
@@ -540,7 +548,9 @@ int tc_block_rows(int M) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return 64;
-    return 128;   // more rows: several blocks of 128 (two accumulators of 128 columns in TMEM)
+    if (M <= 128) return 128;
+    return 256;   // more rows: blocks of 256 (one accumulator of 256 columns in TMEM, one MMA of
+                  // N = 256 per K step, each weight unit dequantized once per 256 rows)
 }
 
 TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
@@ -553,7 +563,7 @@ TcPlan plan_gemm_tc(int M, int N, int K, int group, int sym, int n_sm) {
     if (tiles > kGemvStreamMaxTiles) return pl;
     const long long units = tiles * (K / 128);
     pl.ctas = (int)(units < n_sm ? units : n_sm);
-    pl.slot_w = (uint32_t)((kTcUnitsPerLoad * L.record + 127) & ~127u);
+    pl.slot_w = (uint32_t)((tc_units_per_load(pl.bn) * L.record + 127) & ~127u);
     pl.nd = tc_steps(pl.bn);   // steps in flight: activation tiles in shared memory, weights in TMEM
     pl.na = pl.nd;
     const uint32_t slot_a = (uint32_t)pl.bn * 256u;
@@ -595,6 +605,7 @@ int launch_tc_bn(int bn, const CUtensorMap& map, const TcParams& prm, size_t sme
         case 32: return launch_tc_typed<32, T>(map, prm, smem, stream);
         case 64: return launch_tc_typed<64, T>(map, prm, smem, stream);
         case 128: return launch_tc_typed<128, T>(map, prm, smem, stream);
+        case 256: return launch_tc_typed<256, T>(map, prm, smem, stream);
         default: return W4A16_EUNSUPPORTED;
     }
 }
