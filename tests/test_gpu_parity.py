@@ -305,10 +305,12 @@ def test_gemm_tiled_full_output(M, K, N, group, sym, a_dtype, kernel):
 
 @pytest.mark.parametrize("a_dtype", [0, 1])
 @pytest.mark.parametrize("sym", [0, 1])
-def test_gemm_tc_unit_rows_return_dequantized_rows(a_dtype, sym):
+@pytest.mark.parametrize("reps", [5, 25])
+def test_gemm_tc_unit_rows_return_dequantized_rows(a_dtype, sym, reps):
     K, N, group = 512, 256, 64
     Wb, (oc, os_, oz), tiled = _tiled("normal", K, N, group, sym, 31)
-    rows = [0, 1, 7, 8, 63, 64, 200, 511] * 5   # 40 rows -> the tensor-core path
+    # 40 rows (a 64-row tile, two MMA threads) or 200 rows (a 256-row tile, N = 256 MMAs)
+    rows = [0, 1, 7, 8, 63, 64, 200, 511] * reps
     Ab = np.zeros((len(rows), K), dtype=np.uint16)
     one = 0x3C00 if a_dtype == 0 else 0x3F80
     for i, k in enumerate(rows):
