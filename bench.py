@@ -540,11 +540,10 @@ def bench_naive(torch, native, synthetic, seed, steps, warmup, copies=4):
     return out
 
 
-def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv", "o")):
-    """The calibrated encoders (offline, once per layer), GPTQ and AWQ, on Llama-3-8B decode
-    shapes (by default the two with K = 4096 and N <= 6144, to keep the run short) with S
-    calibration rows (fp16): device time per layer (CUDA events around the whole call), and the
-    layer-output error on the calibration inputs relative to RTN's, ||X W - X' W_hat||^2
+def bench_encoders(torch, native, synthetic, seed, reps=2, S=512, shapes=("qkv", "o", "gate_up", "down")):
+    """The calibrated encoders (offline, once per layer), GPTQ and AWQ, on the Llama-3-8B decode
+    shapes with S calibration rows (fp16): device time per layer (CUDA events around the whole
+    call), and the layer-output error on the calibration inputs relative to RTN's, ||X W - X' W_hat||^2
     (X' = X for GPTQ, X S^-1 for AWQ)."""
     dev = torch.device("cuda")
     out = {}

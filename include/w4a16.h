@@ -148,8 +148,8 @@ W4A16_API size_t w4a16_gptq_workspace_bytes(int K, int N);
  *   X          device, calibration inputs [S, K] row-major, 16-bit of type x_dtype.
  *   x_dtype    W4A16_F16 or W4A16_BF16.
  *   S          calibration rows, >= 1.
- *   K, N, group, sym   as for w4a16_quantize; K <= 29056 (the triangular inverse keeps one FP64
- *              column of K values in shared memory), else W4A16_EUNSUPPORTED.
+ *   K, N, group, sym   as for w4a16_quantize (the workspace, 16 K^2 + 8 K N bytes, is the only
+ *              limit on K).
  *   damp       damping as a fraction of mean(diag H), added to the diagonal (0.01 is usual);
  *              >= 0 and finite.
  *   codes, scales, zeros   device out, the plain layout of w4a16_quantize (zeros NULL iff sym).
@@ -157,7 +157,7 @@ W4A16_API size_t w4a16_gptq_workspace_bytes(int K, int N);
  *              aligned; contents on entry do not matter.
  *   dev_status nullable device int: W4A16_ENONFINITE when W holds Inf/NaN or H + damping is not
  *              positive definite (outputs then unspecified).
- *   stream     cudaStream_t. About 2 K + 2 K / 128 + 4 kernel launches.
+ *   stream     cudaStream_t. About 3 K / 32 + 4 kernel launches.
  * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
  * W4A16_ECUDA (host-side checks; nothing is launched on an error).
  */

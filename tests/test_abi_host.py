@@ -197,8 +197,8 @@ def test_gptq_rejects_bad_arguments_before_any_launch(L):
     assert call(ws=None) == native.EINVAL
     assert call(wsb=need - 1) == native.EWORKSPACE
     assert call(X=P((2 << 20) + 2)) == native.EALIGN
-    big = 29056 + 128
-    assert call(K=big, wsb=L.w4a16_gptq_workspace_bytes(big, N)) == native.EUNSUPPORTED
+    big = 65536   # the factorisations are blocked, so only the workspace grows with K
+    assert L.w4a16_gptq_workspace_bytes(big, N) == 16 * big * big + 8 * big * N + 1024 * N + 256
 
 
 def test_awq_rejects_bad_arguments_before_any_launch(L):

@@ -38,6 +38,7 @@ def _np(t, dt):
     (512, 256, 384, 32, 1, 1),
     (320, 96, 200, 64, 0, 1),     # a ragged last block of 64 channels; S not a multiple of 32
     (384, 264, 512, 128, 1, 0),   # N not a multiple of the 32-channel CTA
+    (352, 64, 300, 32, 0, 0),     # K not a multiple of 64: a ragged last block of the factorisation
 ])
 def test_gptq_bit_exact_full(K, N, S, group, sym, x_dtype):
     Wb = synthetic.weights_normal(K, N, 300 + K)

@@ -149,7 +149,6 @@ W4A16_API int w4a16_gptq_quantize(const void* W, const void* X, int x_dtype, int
     if (!aligned16(W) || !aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
         (zeros && !aligned16(zeros)))
         return W4A16_EALIGN;
-    if ((size_t)K * sizeof(double) > 227 * 1024) return W4A16_EUNSUPPORTED;   // one FP64 column of U in shared memory
     if (ws_bytes < gptq_workspace_bytes(K, N)) return W4A16_EWORKSPACE;
     return launch_gptq(W, X, x_dtype, S, K, N, group, sym, damp, codes, scales, zeros, workspace, dev_status,
                        static_cast<cudaStream_t>(stream));
