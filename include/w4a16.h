@@ -279,10 +279,11 @@ W4A16_API size_t w4a16_workspace_bytes(int M, int N, int K, int group);
  * The environment variable W4A16_FORCE_KERNEL=gemv|tc overrides the choice.
  * On the tiled layout the decode GEMV is the persistent stream-K kernel (one CTA per SM, unit
  * records streamed by bulk copies, warp-level tensor-core MMA). When the M rows of A for the
- * whole K do not fit in its shared memory it runs over S equal slices of K (one launch each,
- * FP32 slice outputs added in order by a last kernel). AUTO takes it for M <= 8 (whole K or
- * slices) and for 9 <= M <= 16 only when K fits whole; otherwise the tensor-core GEMM (measured:
- * with 9-16 rows the sliced decode kernel is slower than the tensor-core GEMM).
+ * whole K do not fit in its shared memory it runs over S equal slices of K (each served by its
+ * own CTAs of one launch, FP32 slice outputs added in order by a last kernel). AUTO takes it for
+ * M <= 8 (whole K or slices) and for 9 <= M <= 16 only when K fits whole; otherwise the
+ * tensor-core GEMM (measured: with 9-16 rows the sliced decode kernel is slower than the
+ * tensor-core GEMM).
  */
 W4A16_API int w4a16_select_kernel(int M, int N, int K, int group);
 

@@ -577,7 +577,8 @@ def test_gemm_llama70b_decode_all_columns(K, N, M):
 @pytest.mark.parametrize("M", [6, 9])
 def test_gemm_auto_sweep_shape_skinny_all_columns(M):
     """M rows of A too long to sit in the decode kernel's shared memory whole: the AUTO dispatch
-    runs the decode kernel over K slices (one launch each, FP32 outputs added in slice order) or
+    runs the decode kernel over K slices (CTA groups of one launch, FP32 outputs added in slice
+    order) or
     the tensor-core kernel, every output within the bound."""
     K, N, group, sym, a_dtype = 8192, 28672, 128, 0, 1
     Wb, (oc, os_, oz), tiled = _tiled("outliers", K, N, group, sym, 6)
@@ -593,8 +594,9 @@ def test_gemm_auto_sweep_shape_skinny_all_columns(M):
     (12, 16384, 8192, 64, 0, 1),    # eight slices of 2048
 ])
 def test_gemm_stream_k_slices_full_output(M, K, N, group, sym, a_dtype):
-    """The decode kernel over K slices: full output within the bound, stages that run across a
-    tile boundary of the slice (two copies), counters left at zero, and a second call identical."""
+    """The decode kernel over K slices, each served by its own CTAs of one launch: full output
+    within the bound, stages that run across a tile boundary of the slice (two copies), every
+    slice's counters left at zero, and a second call identical."""
     kind = "student_t" if sym else "outliers"
     Wb, (oc, os_, oz), tiled = _tiled(kind, K, N, group, sym, 170 + M)
     Ab, A = _acts(M, K, 1700 + M, a_dtype)

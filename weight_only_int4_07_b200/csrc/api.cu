@@ -66,10 +66,10 @@ const char* kernel_name(int k) {
 
 // The dispatch proper (tiled layout), without the environment override. For small M the layer is
 // bound by the weight stream and the stream-K decode GEMV serves it (over K slices when the M rows
-// of A do not fit in its shared memory at once); above, the tensor-core GEMM. Measured on the (8192, 28672), (28672, 8192) and (4096, 28672) layers (bf16, g128): the decode
-// kernel beats the tensor-core GEMM by 2-3x for M <= 8 whether K is held whole or in slices; for
-// M = 9..16 (two 8-row MMA tiles) it wins only when K is held whole, and is up to 1.8x slower when
-// K needs 8 or more slices.
+// of A do not fit in its shared memory at once); above, the tensor-core GEMM. Measured on the
+// (8192, 28672), (28672, 8192) and (4096, 28672) layers (bf16, g128): for M <= 8 the decode kernel
+// beats the tensor-core GEMM (1.2-1.6x) whether K is held whole or in slices; for M = 9..16 (two
+// 8-row MMA tiles) it wins only when K is held whole, and is 1.7-2.2x slower when K needs slices.
 int dispatch(int M, int N, int K, int group) {
     if (M > 16) return W4A16_KERNEL_TC;
     if (M <= 8) return W4A16_KERNEL_GEMV;

@@ -88,10 +88,10 @@ constexpr int kGemvStreamMaxTiles = (int)(kGemvStreamCounterBytes / 4);
 struct GemvStreamPlan {
     bool ok;
     int ns;               // pipeline stages
-    int ctas;             // persistent CTAs (one per SM)
+    int ctas;             // persistent CTAs of each slice (one per SM in all)
     size_t row_bytes, act_bytes, red_bytes, sa_bytes, stage_bytes, smem;
     size_t partial_bytes; // workspace after the counters (cut-tile sums, then the slices' outputs)
-    int slices;           // launches over equal K slices (1: the whole K at once)
+    int slices;           // equal K slices, each served by its own CTAs (1: the whole K at once)
 };
 GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm);
 int gemv_stream_sm_count();
@@ -104,7 +104,7 @@ struct TcPlan {
     bool ok;
     int bn;               // rows of A per tile (the MMA's N)
     int mblocks;          // tiles of BN rows
-    int ctas;             // persistent CTAs (one per SM)
+    int ctas;             // persistent CTAs of each slice (one per SM in all)
     int nr, na, nd;       // ring depths: record slots, activation tiles, weight tiles
     uint32_t slot_w, off_a, off_w, off_bar;
     size_t smem;

@@ -105,10 +105,11 @@ struct GsParams {
     uint32_t stage_bytes, row_bytes, act_bytes, red_bytes, sa_bytes;
     GsMasks km;
     GsMasks km_native;   // bf16 masks, for bf16 rows kept in bf16 at group 128
-    // K slice of this launch: A points at its first column, rows lda elements apart; the slice's
-    // units are K-steps c0 .. c0 + K/128 of every tile of a K_total/128 = ktot-step weight; with
-    // out_f32 set the FP32 sums go there ([M][N]) instead of C
-    int lda, c0, ktot;
+    // K slices: K is the width of one slice, A points at the first column of slice 0, rows lda
+    // elements apart; slice sl covers the K-steps c0 + sl K/128 .. of every tile of a
+    // ktot-step weight and is served by CTAs sl P .. sl P + P - 1 of the grid (slices x P CTAs);
+    // with out_f32 set the FP32 sums of slice sl go to out_f32 + sl M N ([M][N]) instead of C
+    int lda, c0, ktot, slices;
     float* out_f32;
     uint64_t wait_ns;   // limit of every bounded wait (the drain after a timeout keeps kGsSpin)
 };
@@ -134,7 +135,15 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const int M = p.M, K = p.K, N = p.N, ns = p.ns, P = p.P;
     const int steps = K / 128;
     const long long U = (long long)(N / 128) * steps;
-    const int cta = blockIdx.x;
+    // K slices fused into one launch: CTAs [sl P, sl P + P) serve slice sl, i.e. columns
+    // sl K .. sl K + K - 1 of A and weight steps c0 + sl K/128 .., with their own tile counters and
+    // partial sums, and FP32 sums to out_f32 + sl M N (a single slice: sl = 0)
+    const int sl = (int)blockIdx.x / P;
+    const int cta = (int)blockIdx.x - sl * P;
+    const int kc0 = p.c0 + sl * steps;
+    int* const counters = p.counters + sl * (N / 128);
+    float* const partials = p.partials + (size_t)sl * P * M * 128;
+    float* const out_f32 = p.out_f32 ? p.out_f32 + (size_t)sl * M * N : nullptr;
     const long long u0 = unit_begin(cta, U, P), u1 = unit_begin(cta + 1, U, P);
     const int nunits = (int)(u1 - u0);
     const uint32_t R = p.record, stage_bytes = p.stage_bytes, RS = p.row_bytes;
@@ -190,9 +199,9 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
             const long long t = ua / steps;
             const int cc = (int)(ua - t * steps);
             const int n1 = steps - cc < n ? steps - cc : n;
-            bulk_g2s(dst, p.tiled + ((size_t)t * p.ktot + p.c0 + cc) * R, (uint32_t)n1 * R, &full[s]);
+            bulk_g2s(dst, p.tiled + ((size_t)t * p.ktot + kc0 + cc) * R, (uint32_t)n1 * R, &full[s]);
             if (n1 < n)
-                bulk_g2s(dst + (size_t)n1 * R, p.tiled + ((size_t)(t + 1) * p.ktot + p.c0) * R, (uint32_t)(n - n1) * R,
+                bulk_g2s(dst + (size_t)n1 * R, p.tiled + ((size_t)(t + 1) * p.ktot + kc0) * R, (uint32_t)(n - n1) * R,
                          &full[s]);
         }
         ++issued[s];
@@ -205,7 +214,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     const int grp = warp / kGsGroupWarps, wg = warp % kGsGroupWarps;
     const int g = lane >> 2, t = lane & 3;
     const int ch0 = 32 * wg + g;     // this lane's channels: ch0 + 8 r, r = 0..3
-    const T* A = static_cast<const T*>(p.A);
+    const T* A = static_cast<const T*>(p.A) + (size_t)sl * K;
 
     bool wide = false;   // kConv: some row keeps bf16 values and the bf16 arithmetic
 
@@ -557,7 +566,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                     const uint64_t t0 = globaltimer_ns();
                     for (;;) {
                         int n;
-                        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(p.counters + etile)
+                        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(n) : "l"(counters + etile)
                                      : "memory");
                         if (n >= cl - cf) break;
                         if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
@@ -566,7 +575,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                             break;
                         }
                     }
-                    p.counters[etile] = 0;
+                    counters[etile] = 0;
                 }
                 __syncwarp();
                 for (int m = 0; m < M; ++m) {
@@ -578,7 +587,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                         for (int q = 0; q < 4; ++q)
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
-                                ld[q][j] = c0 + q <= cl ? __ldcg(p.partials + ((size_t)(c0 + q) * M + m) * 128 + lane + 32 * j)
+                                ld[q][j] = c0 + q <= cl ? __ldcg(partials + ((size_t)(c0 + q) * M + m) * 128 + lane + 32 * j)
                                                         : 0.0f;
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -605,8 +614,8 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                         float o = (rb[(0 * M + m) * 128 + ch] + rb[(1 * M + m) * 128 + ch] + rb[(2 * M + m) * 128 + ch] +
                                    rb[(3 * M + m) * 128 + ch]) * up;
                         if (gather) o += pre[m * 128 + ch];
-                        if (p.out_f32)
-                            p.out_f32[(size_t)m * N + n0 + ch] = o;
+                        if (out_f32)
+                            out_f32[(size_t)m * N + n0 + ch] = o;
                         else
                             C[(size_t)m * N + n0 + ch] = Act<T>::from_f32(o);
                     }
@@ -614,7 +623,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
             } else {
                 // a later CTA of a cut tile (the tile opens its range): publish this CTA's sums and
                 // count them, without waiting
-                float* part = p.partials + (size_t)cta * M * 128;
+                float* part = partials + (size_t)cta * M * 128;
                 for (int m = 0; m < M; ++m) {
                     float up = 1.0f;
                     if constexpr (kConv)   // undo the row's 2^-k (this CTA's)
@@ -629,7 +638,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
                 __threadfence();
                 __syncwarp();
                 if (lane == 0)
-                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.counters + etile) : "memory");
+                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counters + etile) : "memory");
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[bsel]);
@@ -710,7 +719,7 @@ int launch_typed(const GsParams& prm, size_t smem, cudaStream_t stream) {
     });
     if (attr_err != cudaSuccess) return W4A16_ECUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(prm.P, 1, 1);
+    cfg.gridDim = dim3(prm.P * prm.slices, 1, 1);
     cfg.blockDim = dim3(kGsThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -794,16 +803,17 @@ GemvStreamPlan plan_slice(int M, int N, int Ks, int group, int sym, int n_sm) {
 
 }  // namespace
 
-// The whole K in one launch when the M rows of A fit in shared memory beside three stages;
-// otherwise K is cut into S equal slices (S a power of two dividing K / 128), one launch each,
-// whose FP32 outputs a last kernel adds in slice order.
+// The whole K at once when the M rows of A fit in shared memory beside three stages; otherwise K
+// is cut into S equal slices (S a power of two dividing K / 128), each served by its own group of
+// n_sm / S CTAs of the same launch, whose FP32 outputs a last kernel adds in slice order.
 GemvStreamPlan plan_gemv_stream(int M, int N, int K, int group, int sym, int n_sm) {
     GemvStreamPlan pl = {};
     if (M < 1 || M > 16 || K % 128 != 0 || N % 128 != 0 || K < 128 || N < 128) return pl;
     if (group != 32 && group != 64 && group != 128) return pl;
     if (N / 128 > kGemvStreamMaxTiles) return pl;
     for (int S = 1; S <= 64 && (K / 128) % S == 0; S *= 2) {
-        pl = plan_slice(M, N, K / S, group, sym, n_sm);
+        if ((long long)(N / 128) * S > kGemvStreamMaxTiles) break;   // tile counters of every slice
+        pl = plan_slice(M, N, K / S, group, sym, S > 1 ? n_sm / S : n_sm);
         if (pl.ok) {
             pl.slices = S;
             pl.partial_bytes = (size_t)2 * kGsCtasPerSm * (n_sm > 0 ? n_sm : 0) * M * 128 * 4 +
@@ -859,14 +869,13 @@ int launch_gemv_stream(const void* A, int a_dtype, int M, int K, const void* til
     prm.km_native = prm.km;
     prm.km_native.hi = 0x000F000Fu;
     prm.km_native.magic = 0x43004300u;
-    for (int sl = 0; sl < S; ++sl) {
-        prm.A = static_cast<const uint16_t*>(A) + (size_t)sl * Ks;
-        prm.c0 = sl * (Ks / 128);
-        prm.out_f32 = S > 1 ? slice_out + (size_t)sl * M * N : nullptr;
-        const int st = bf16 ? launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream)
-                            : launch_rows<__half>(prm, group, pl.smem, stream);
-        if (st != W4A16_OK) return st;
-    }
+    prm.A = A;
+    prm.c0 = 0;
+    prm.slices = S;
+    prm.out_f32 = S > 1 ? slice_out : nullptr;
+    const int st = bf16 ? launch_rows<__nv_bfloat16>(prm, group, pl.smem, stream)
+                        : launch_rows<__half>(prm, group, pl.smem, stream);
+    if (st != W4A16_OK) return st;
     if (S > 1) {
         const size_t MN = (size_t)M * N;
         const unsigned blocks = (unsigned)((MN + 255) / 256 < 2048 ? (MN + 255) / 256 : 2048);
