@@ -115,7 +115,9 @@ struct GsParams {
 };
 
 // NB: n8 tiles of activation rows (1: M <= 8, 2: M <= 16). ODD: rows 2t + 1 of an n8 tile exist.
-template <int NB, typename T, int GROUP, bool ODD>
+// SL: the launch serves several K slices (a separate instance, so that the single-slice one keeps
+// no slice arithmetic).
+template <int NB, typename T, int GROUP, bool ODD, bool SL>
 __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(const GsParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     constexpr bool kPost = (GROUP == 128);   // one group per unit: scale the unit's sum
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     // K slices fused into one launch: CTAs [sl P, sl P + P) serve slice sl, i.e. columns
     // sl K .. sl K + K - 1 of A and weight steps c0 + sl K/128 .., with their own tile counters and
     // partial sums, and FP32 sums to out_f32 + sl M N (a single slice: sl = 0)
-    const int sl = (int)blockIdx.x / P;
+    const int sl = SL ? (int)blockIdx.x / P : 0;
     const int cta = (int)blockIdx.x - sl * P;
     const int kc0 = p.c0 + sl * steps;
     int* const counters = p.counters + sl * (N / 128);
@@ -709,12 +711,12 @@ __global__ void __launch_bounds__(kGsThreads, kGsCtasPerSm) gemv_stream_kernel(c
     }
 }
 
-template <int NB, typename T, int GROUP, bool ODD>
+template <int NB, typename T, int GROUP, bool ODD, bool SL>
 int launch_typed(const GsParams& prm, size_t smem, cudaStream_t stream) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<NB, T, GROUP, ODD>,
+        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<NB, T, GROUP, ODD, SL>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGsSmemMax);
     });
     if (attr_err != cudaSuccess) return W4A16_ECUDA;
@@ -728,25 +730,31 @@ int launch_typed(const GsParams& prm, size_t smem, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_stream_kernel<NB, T, GROUP, ODD>, prm);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_stream_kernel<NB, T, GROUP, ODD, SL>, prm);
     return e == cudaSuccess ? W4A16_OK : W4A16_ECUDA;
 }
 
-template <int NB, typename T, bool ODD>
+template <int NB, typename T, bool ODD, bool SL>
 int launch_group(const GsParams& prm, int group, size_t smem, cudaStream_t stream) {
     switch (group) {
-        case 32: return launch_typed<NB, T, 32, ODD>(prm, smem, stream);
-        case 64: return launch_typed<NB, T, 64, ODD>(prm, smem, stream);
-        case 128: return launch_typed<NB, T, 128, ODD>(prm, smem, stream);
+        case 32: return launch_typed<NB, T, 32, ODD, SL>(prm, smem, stream);
+        case 64: return launch_typed<NB, T, 64, ODD, SL>(prm, smem, stream);
+        case 128: return launch_typed<NB, T, 128, ODD, SL>(prm, smem, stream);
         default: return W4A16_EUNSUPPORTED;
     }
 }
 
+template <int NB, typename T, bool ODD>
+int launch_sliced(const GsParams& prm, int group, size_t smem, cudaStream_t stream) {
+    return prm.slices > 1 ? launch_group<NB, T, ODD, true>(prm, group, smem, stream)
+                          : launch_group<NB, T, ODD, false>(prm, group, smem, stream);
+}
+
 template <typename T>
 int launch_rows(const GsParams& prm, int group, size_t smem, cudaStream_t stream) {
-    if (prm.M > 8) return launch_group<2, T, true>(prm, group, smem, stream);
-    if (prm.M > 1) return launch_group<1, T, true>(prm, group, smem, stream);
-    return launch_group<1, T, false>(prm, group, smem, stream);
+    if (prm.M > 8) return launch_sliced<2, T, true>(prm, group, smem, stream);
+    if (prm.M > 1) return launch_sliced<1, T, true>(prm, group, smem, stream);
+    return launch_sliced<1, T, false>(prm, group, smem, stream);
 }
 
 // C = sum over the S slices of the FP32 partial outputs, in slice order.
