@@ -42,7 +42,7 @@ constexpr int kGptqWarps = 8;       // warps of the block kernel (each owns ever
 constexpr int kGptqThreads = 32 * kGptqWarps;   // block kernel: 32 output channels per CTA
 constexpr int kTrailTile = 64;      // trailing GEMM output tile (rows x columns)
 constexpr int kTrailK = 16;         // trailing GEMM k-chunk
-constexpr int kCholBlock = 64;      // panel width of the blocked factorisations
+constexpr int kCholBlock = 64;      // leaf block and tile size of the recursive factorisation
 constexpr int kCP = kCholBlock + 1; // padded shared-memory row pitch (doubles)
 constexpr int kCholK = 16;          // k-chunk of the tiled products
 
