@@ -54,6 +54,23 @@ def test_step_time_model_reproduces_the_worked_example():
         assert _digits(t * 1e3, ms) == ms
 
 
+def test_decode_traffic_record_applies_only_to_its_sources(tmp_path, monkeypatch):
+    """The ncu traffic record behind `roofline.traffic`: scaled to a launch's algorithmic bytes
+    while its source hash matches the decode kernel's sources, null (stale) once they differ."""
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    assert {"sources_sha", "dram_bytes", "algorithmic_bytes", "capture"} <= set(rec)
+    assert 1.0 <= rec["dram_bytes"] / rec["algorithmic_bytes"] < 1.1   # each unit record read once
+    path = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    path.write_text(json.dumps(dict(rec, sources_sha=bench.decode_sources_sha())))
+    b, info = bench.decode_traffic(3 * rec["algorithmic_bytes"])
+    assert b == pytest.approx(3 * rec["dram_bytes"])
+    assert info["ratio_to_algorithmic"] == pytest.approx(rec["dram_bytes"] / rec["algorithmic_bytes"])
+    path.write_text(json.dumps(dict(rec, sources_sha="0" * 16)))
+    b, info = bench.decode_traffic(1e8)
+    assert b is None and info["stale"]
+
+
 def test_algorithmic_bytes_match_the_format():
     """0.515625 byte/weight for g128 with an FP16 scale; + 0.5/128 with INT4 zero-points."""
     K, N = 4096, 4096
