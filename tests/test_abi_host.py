@@ -247,6 +247,19 @@ def test_workspace_covers_the_k_slices_of_the_decode_kernel():
     assert native.w4a16_workspace_bytes(M, N, K, 128) >= 65536 + 2 * M * N * 4
     # one row fits whole: counters plus the cut-tile sums only
     assert native.w4a16_workspace_bytes(1, N, K, 128) < 65536 + M * N * 4
+    # 8 rows: two slices of 4096, served by the two CTA groups of one launch
+    assert native.w4a16_workspace_bytes(8, N, K, 128) >= 65536 + 2 * 8 * N * 4
+
+
+@pytest.mark.parametrize("K,N", [(8192, 28672), (8192, 10240), (8192, 57344), (28672, 8192), (4096, 28672)])
+def test_dispatch_on_the_benchmarked_layers(K, N):
+    """The sweep layer and the 70B and 8B layers (bf16, g128): the decode GEMV up to 8 rows, whole
+    K or sliced; from 9 rows the tensor-core GEMM, since 9-16 rows of these K need K slices, where
+    the decode kernel's two 8-row MMA tiles make it slower than the tensor-core GEMM."""
+    for M in range(1, 9):
+        assert native.w4a16_select_kernel(M, N, K, 128) == native.KERNEL_GEMV
+    for M in (9, 12, 16, 17, 64, 256):
+        assert native.w4a16_select_kernel(M, N, K, 128) == native.KERNEL_TC
 
 
 def test_wait_limit_setter_is_host_only(L):
