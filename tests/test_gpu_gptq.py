@@ -71,6 +71,21 @@ def test_gptq_bit_exact_sampled_columns():
     assert np.array_equal(gzw[:, [0, 256]], oz)
 
 
+def test_gptq_bit_exact_sampled_columns_deep_factorisation():
+    """K = 4096 (64 blocks of 64 channels: six levels of the recursive factorisation), symmetric,
+    group 64, bf16 calibration rows; 16 sampled output channels, among them the last CTA's, agree
+    with the oracle bit for bit."""
+    K, N, S, group, sym = 4096, 4096, 1024, 64, 1
+    Wb = synthetic.weights_outliers(K, N, 312)
+    Xb = synthetic.calibration(S, K, 313, dtype=synthetic.BF16)
+    gc, gs, _ = native.w4a16_gptq_quantize(_dev16(Wb, synthetic.F16), _dev16(Xb, synthetic.BF16), group, sym)
+    torch.cuda.synchronize()
+    cols = np.r_[8:16, 4080:4088]
+    oc, os_, _ = ogptq.gptq(np.ascontiguousarray(Wb[:, cols]), Xb, synthetic.BF16, group, sym)
+    assert np.array_equal(_np(gc, np.int32)[:, cols], oc)
+    assert np.array_equal(_np(gs.view(torch.int16), np.uint16)[:, cols], os_)
+
+
 @pytest.mark.parametrize("sym", [0, 1])
 def test_gptq_lowers_output_error_at_layer_size(sym):
     """The 8B o-proj shape (4096 x 4096) with 512 calibration rows: GPTQ's layer-output error on
