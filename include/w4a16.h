@@ -157,7 +157,7 @@ W4A16_API size_t w4a16_gptq_workspace_bytes(int K, int N);
  *              aligned; contents on entry do not matter.
  *   dev_status nullable device int: W4A16_ENONFINITE when W holds Inf/NaN or H + damping is not
  *              positive definite (outputs then unspecified).
- *   stream     cudaStream_t. About 3 K / 32 + 4 kernel launches.
+ *   stream     cudaStream_t. About 3 K / 32 kernel launches.
  * Returns W4A16_OK, W4A16_EINVAL, W4A16_EALIGN, W4A16_EUNSUPPORTED, W4A16_EWORKSPACE or
  * W4A16_ECUDA (host-side checks; nothing is launched on an error).
  */
